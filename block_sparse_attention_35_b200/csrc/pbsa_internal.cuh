@@ -1,0 +1,85 @@
+// pbsa_internal.cuh - host-side geometry and kernel launcher declarations shared by the
+// PBSA translation units (not part of the public ABI).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "pbsa.h"
+
+namespace pbsa {
+
+// Geometry derived from a pbsa_config (all counts in tokens, blocks or frames).
+struct Geo {
+    int B, H, D;
+    int fh, fw, tf;     // frame grid and tokens per frame
+    int nby, nbx, nbf;  // block rows, block columns, blocks per frame
+    int W;              // frame slots of the local ring
+    int S;              // persistent slots
+};
+
+// Forward-pass launch arguments.
+struct FwdArgs {
+    Geo g;
+    int q_frames, local_frames, ring_head;
+    int idx_stride;
+    int ucap;            // capacity of the per-tile union of selections
+    int n_seg_max;       // mass segments per CTA (S + ucap)
+    const int32_t* pers_len;
+    const int32_t* idx;
+    const int32_t* cnt;
+    float* lse;
+    float* mass_local;
+    float* mass_pers;
+    float* scratch;      // mass partials, [ctas][n_seg_max][128]
+    int32_t* status;
+    CUtensorMap tm_q, tm_o, tm_kl, tm_vl, tm_kp, tm_vp;
+};
+
+// Backward-pass launch arguments.
+struct BwdArgs {
+    Geo g;
+    int q_frames, local_frames, ring_head;
+    int idx_stride;
+    const int32_t* pers_len;
+    const int32_t* idx;
+    const int32_t* cnt;
+    const float* lse;
+    const __nv_bfloat16* out;
+    const __nv_bfloat16* dout;
+    float* delta;        // [B, H, Nq] workspace
+    float* dq;
+    float* dk_pers;
+    float* dv_pers;
+    float* dk_local;
+    float* dv_local;
+    int32_t* status;
+    CUtensorMap tm_q, tm_do, tm_kl, tm_vl, tm_kp, tm_vp;
+};
+
+// Launchers (return a cudaError_t from the launch).
+cudaError_t launch_pool(const Geo& g, const __nv_bfloat16* q, int q_frames,
+                        const __nv_bfloat16* k_local, int local_frames, int ring_head,
+                        float* qbar, float* kbar, cudaStream_t st);
+cudaError_t launch_score_topk(const Geo& g, const float* qbar, const float* kbar, int qb,
+                              int nl, int k, int32_t* idx, int idx_stride, int32_t* cnt,
+                              float* scores, cudaStream_t st);
+size_t score_topk_smem_bytes(const Geo& g, int nl);
+
+cudaError_t launch_attn_fwd(const FwdArgs& a, bool with_mass, cudaStream_t st);
+size_t attn_fwd_smem_bytes(const Geo& g, int ucap);
+
+cudaError_t launch_attn_bwd(const BwdArgs& a, cudaStream_t st);
+
+cudaError_t launch_cache_update(const Geo& g, const __nv_bfloat16* k_local,
+                                const __nv_bfloat16* v_local, int local_frames, int ring_head,
+                                float* mass_local, int n_evict_frames, int first_frame_global,
+                                __nv_bfloat16* k_pers, __nv_bfloat16* v_pers, int32_t* pers_len,
+                                float* pers_score, int32_t* pers_src, int32_t* upd,
+                                int32_t* n_upd, cudaStream_t st);
+
+cudaError_t launch_wait_selftest(int32_t* status, long long timeout_ns, cudaStream_t st);
+
+}  // namespace pbsa

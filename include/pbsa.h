@@ -1,0 +1,231 @@
+/*
+ * pbsa.h - C ABI of the Persistent Block-Sparse Attention (PBSA) library, NVIDIA B200
+ * (sm_100a).
+ *
+ * PBSA is the attention of "Sparse Forcing: Native Trainable Sparse Attention for
+ * Real-time Autoregressive Diffusion Video Generation" (pith.science, abstract): a chunk of
+ * video query tokens attends to every block of a persistent cache and to a top-k
+ * selection of the 1x8x8 token blocks of a sliding local window; when the window slides,
+ * the evicted blocks are merged into the persistent cache.  The argument names follow the
+ * project page's usage snippet of SparseForcingAttention (boxunxu.top/SparseForcing):
+ * total_cache_size, local_cache_size, persistent_cache_size, kv_cache_mode,
+ * sparse_kv_block_size, max_seq_len, use_local_block_sparse_attn,
+ * local_block_sparse_topk_ratio, and the call attn(query, key_persistent,
+ * value_persistent, key_local, value_local).
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - Every tensor pointer is a DEVICE pointer owned by the caller.  The library never
+ *    allocates or frees device memory; scratch comes from the caller's `workspace`
+ *    (size from pbsa_workspace_size).  Pointers must be 16-byte aligned.
+ *  - `stream` is a cudaStream_t passed as void*.  Every call is asynchronous on it and
+ *    performs no host synchronisation.
+ *  - Return value: PBSA_OK (0) or a negative PBSA_ERR_* code.  Argument errors are found
+ *    on the host before anything is launched; pbsa_last_error() then gives a message
+ *    (thread-local, valid until the next call on the same thread).
+ *  - `status` (where present) is a device int32 the caller zeroes; kernels write
+ *    PBSA_ERR_TIMEOUT into it when a bounded wait runs out (the kernel then returns
+ *    early and its outputs are undefined) and PBSA_ERR_DEVICE_CHECK when an index read
+ *    from device memory is out of range (the bad entry is skipped).
+ *  - Layouts (B batch, H heads, D head dim, T_f = frame_h * frame_w tokens per frame,
+ *    tokens of a frame in raster order n = y * frame_w + x, frames consecutive):
+ *      query / out           [B, q_frames * T_f, H, D]      bf16
+ *      key_local/value_local [B, W * T_f, H, D]              bf16, a ring of W =
+ *                            local_cache_size / T_f frame slots.  The window holds
+ *                            `local_frames` frames; its frame p (0 = oldest) lives in
+ *                            ring slot (ring_head + p) % W.
+ *      key_persistent / value_persistent [B, H, S, 64, D]   bf16: S slots of one block
+ *                            each, the block's tokens in raster order in rows
+ *                            0 .. pers_len-1 (rows past pers_len are ignored).
+ *      pers_len [B, H, S] int32 (0 = empty slot, else the block's token count, a
+ *                            multiple of 8 for 8x8 blocks cut by the frame edge).
+ *  - Blocks: 1 x 8 x 8 tokens; a frame has NB_f = ceil(frame_h/8) * ceil(frame_w/8)
+ *    blocks numbered by * ceil(frame_w/8) + bx; edge blocks are clipped to the frame.
+ *    Local block ids are LOGICAL: window frame p, block i -> p * NB_f + i.  Query block
+ *    ids: chunk frame f, block i -> f * NB_f + i.
+ */
+#ifndef PBSA_H
+#define PBSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define PBSA_API __attribute__((visibility("default")))
+#else
+#define PBSA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define PBSA_OK 0
+#define PBSA_ERR_ARG (-1)          /* bad argument: null pointer, size, alignment */
+#define PBSA_ERR_UNSUPPORTED (-2)  /* valid per the pages but not built here */
+#define PBSA_ERR_CUDA (-3)         /* a CUDA runtime/driver call failed */
+#define PBSA_ERR_TIMEOUT (-4)      /* device status: a bounded wait ran out */
+#define PBSA_ERR_DEVICE_CHECK (-5) /* device status: an index was out of range */
+#define PBSA_ERR_WORKSPACE (-6)    /* workspace too small */
+
+#define PBSA_KV_CACHE_SPARSE_FORCING 0 /* kv_cache_mode="sparse_forcing" */
+
+/* Operation ids for pbsa_workspace_size. */
+#define PBSA_OP_SELECT 0
+#define PBSA_OP_FWD 1
+#define PBSA_OP_BWD 2
+#define PBSA_OP_UPDATE 3
+
+/*
+ * Configuration: the constructor arguments of SparseForcingAttention (project page,
+ * usage snippet) plus the shapes the pages leave implicit (batch, heads, head dim and
+ * the token grid of a frame).
+ */
+typedef struct pbsa_config {
+    int B, H, D;                 /* batch, heads, head dim (64 or 128) */
+    int frame_h, frame_w;        /* token grid of one frame, e.g. 30 x 52 */
+    int block_t, block_h, block_w; /* sparse_kv_block_size; only {1, 8, 8} is built */
+    int total_cache_size;        /* tokens; must equal local + persistent */
+    int local_cache_size;        /* tokens; a whole number of frames */
+    int persistent_cache_size;   /* tokens */
+    int max_seq_len;             /* tokens; bounds q_frames * T_f */
+    int kv_cache_mode;           /* PBSA_KV_CACHE_SPARSE_FORCING */
+    int use_local_block_sparse_attn; /* 0: every local block is attended */
+    float local_block_sparse_topk_ratio; /* in (0, 1] */
+} pbsa_config;
+
+/* ---------------------------------------------------------------- host-only queries */
+
+/* Checks a configuration; PBSA_OK or an error code (message in pbsa_last_error()). */
+PBSA_API int pbsa_validate_config(const pbsa_config* cfg);
+/* NB_f, blocks per frame. */
+PBSA_API int pbsa_blocks_per_frame(const pbsa_config* cfg);
+/* W, frame slots of the local ring (local_cache_size / T_f). */
+PBSA_API int pbsa_window_frames(const pbsa_config* cfg);
+/* S, persistent slots: persistent_cache_size / T_f * NB_f when that divides, else
+ * ceil(persistent_cache_size / 64). */
+PBSA_API int pbsa_num_slots(const pbsa_config* cfg);
+/* k, local blocks attended per query block for a window of local_frames frames:
+ * N_L = local_frames * NB_f; k = N_L when use_local_block_sparse_attn is 0, else
+ * clamp(ceil(ratio * N_L), 1, N_L). */
+PBSA_API int pbsa_topk_count(const pbsa_config* cfg, int local_frames);
+/* Workspace bytes needed by operation `op` (PBSA_OP_*) for a chunk of q_frames frames. */
+PBSA_API size_t pbsa_workspace_size(const pbsa_config* cfg, int op, int q_frames);
+/* Message of the last error on this thread ("" if none). */
+PBSA_API const char* pbsa_last_error(void);
+/* Library version string. */
+PBSA_API const char* pbsa_version(void);
+
+/* ------------------------------------------------------------------ device calls */
+
+/*
+ * Block selection: the top-k local blocks for every query block.
+ * (pith.science abstract: computation inside each local window is restricted to a
+ * dynamically selected neighbourhood; project page: learned top-k selection with
+ * local_block_sparse_topk_ratio.)
+ *
+ * Score of query block b and local block j: mean of b's valid query tokens . mean of j's
+ * valid key tokens / sqrt(D).  The k best (score descending, then lower logical id) are
+ * written to idx[b] in ascending id order; cnt[b] = k.
+ *
+ *   q        [B, q_frames*T_f, H, D] bf16
+ *   k_local  ring [B, W*T_f, H, D] bf16; window = local_frames frames from ring_head
+ *   idx      [B, H, q_frames*NB_f, idx_stride] int32 out (idx_stride >= k)
+ *   cnt      [B, H, q_frames*NB_f] int32 out
+ *   scores   nullable; [B, H, q_frames*NB_f, local_frames*NB_f] fp32 out
+ *   workspace >= pbsa_workspace_size(cfg, PBSA_OP_SELECT, q_frames) bytes
+ */
+PBSA_API int pbsa_select_blocks(const pbsa_config* cfg, const void* q, int q_frames,
+                       const void* k_local, int local_frames, int ring_head,
+                       int32_t* idx, int idx_stride, int32_t* cnt, float* scores,
+                       void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * PBSA forward.  (pith.science abstract; project page call attn(query, key_persistent,
+ * value_persistent, key_local, value_local).)
+ *
+ * Each query token of query block b attends, with softmax scale 1/sqrt(D), to every valid
+ * row of every occupied persistent slot and to the valid tokens of the local blocks
+ * idx[b][0 .. cnt[b]).
+ *
+ *   out        [B, q_frames*T_f, H, D] bf16 out
+ *   lse        [B, H, q_frames*T_f] fp32 out, natural-log softmax normaliser per row
+ *   mass_local nullable; [B, H, W*NB_f] fp32, indexed by PHYSICAL block
+ *              (ring slot * NB_f + block in frame).  Accumulated (+=): the softmax
+ *              probability summed over this chunk's query rows, per local block.
+ *   mass_pers  nullable; [B, H, S] fp32, accumulated the same way per persistent slot.
+ *              This is the pers_score array of pbsa_cache_update.
+ *   workspace  needed only when a mass output is given:
+ *              >= pbsa_workspace_size(cfg, PBSA_OP_FWD, q_frames) bytes
+ *   status     device int32 (see conventions)
+ */
+PBSA_API int pbsa_attn_fwd(const pbsa_config* cfg, const void* q, int q_frames,
+                  const void* k_pers, const void* v_pers, const int32_t* pers_len,
+                  const void* k_local, const void* v_local, int local_frames, int ring_head,
+                  const int32_t* idx, int idx_stride, const int32_t* cnt,
+                  void* out, float* lse, float* mass_local, float* mass_pers,
+                  void* workspace, size_t workspace_bytes, int32_t* status, void* stream);
+
+/*
+ * PBSA backward (project page: full gradient support for training).  Gradients of
+ * sum(out * dout) with the selection idx held fixed (no gradient flows into the block
+ * scores).  Inputs are the forward's inputs plus its out and lse.
+ *
+ *   dout      [B, q_frames*T_f, H, D] bf16
+ *   dq        [B, q_frames*T_f, H, D] fp32 out (overwritten)
+ *   dk_pers, dv_pers  [B, H, S, 64, D] fp32 out; rows < pers_len overwritten, others
+ *             untouched
+ *   dk_local, dv_local  ring [B, W*T_f, H, D] fp32 out; tokens of the window's frames
+ *             overwritten (0 where no query attended), other ring slots untouched
+ *   workspace >= pbsa_workspace_size(cfg, PBSA_OP_BWD, q_frames) bytes
+ */
+PBSA_API int pbsa_attn_bwd(const pbsa_config* cfg, const void* q, int q_frames,
+                  const void* k_pers, const void* v_pers, const int32_t* pers_len,
+                  const void* k_local, const void* v_local, int local_frames, int ring_head,
+                  const int32_t* idx, int idx_stride, const int32_t* cnt,
+                  const void* out, const float* lse, const void* dout,
+                  float* dq, float* dk_pers, float* dv_pers, float* dk_local,
+                  float* dv_local, void* workspace, size_t workspace_bytes,
+                  int32_t* status, void* stream);
+
+/*
+ * Window slide and persistent merge (pith.science abstract: persistent blocks are
+ * compressed, preserved and updated; algorithm fragment: the t=0 pass updates P and L).
+ *
+ * The oldest n_evict_frames frames of the window leave it.  Candidates are the occupied
+ * slots (score pers_score) followed by the evicted blocks in logical id order (score
+ * mass_local of their physical block).  Ordered by score descending, ties by that
+ * candidate order, the first min(S, #candidates) are kept.  Kept slots stay in place;
+ * the free slots (empty ones ascending, then dropped ones ascending) receive the kept
+ * evicted blocks in id order: tokens copied in raster order, pers_len = token count,
+ * pers_score = the block's mass, pers_src = global frame * NB_f + block in frame, where
+ * the oldest window frame has global number first_frame_global.  Dropped slots that
+ * receive nothing become empty (len 0, score 0, src -1).  The evicted blocks'
+ * mass_local entries are reset to 0.  The caller then advances its ring:
+ * ring_head = (ring_head + n_evict_frames) % W, local_frames -= n_evict_frames.
+ *
+ *   upd    [B, H, n_evict_frames*NB_f, 2] int32 out: (slot, logical block id) per
+ *          admission, in admission order
+ *   n_upd  [B, H] int32 out: admissions per (b, h)
+ *   workspace >= pbsa_workspace_size(cfg, PBSA_OP_UPDATE, 0) bytes
+ */
+PBSA_API int pbsa_cache_update(const pbsa_config* cfg, const void* k_local, const void* v_local,
+                      int local_frames, int ring_head, float* mass_local,
+                      int n_evict_frames, int first_frame_global,
+                      void* k_pers, void* v_pers, int32_t* pers_len, float* pers_score,
+                      int32_t* pers_src, int32_t* upd, int32_t* n_upd,
+                      void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Diagnostic: runs one kernel that waits, with the library's bounded wait, on a barrier
+ * that nothing completes.  After `timeout_ns` nanoseconds the wait gives up and writes
+ * PBSA_ERR_TIMEOUT into *status.  The pages have no counterpart; it exists so that the
+ * timeout path can be tested without hanging a GPU.
+ */
+PBSA_API int pbsa_wait_selftest(int32_t* status, long long timeout_ns, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PBSA_H */

@@ -1,0 +1,151 @@
+"""GPU parity: block selection and the PBSA forward (with block mass) through the C ABI
+against the fp64 oracle on the same seeded inputs."""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+from block_sparse_attention_35_b200 import pbsa as P
+from block_sparse_attention_35_b200.synth import WORKLOADS, Workload, decode_inputs
+from oracle import pbsa_oracle as orc
+from tests.harness import (LSE_ABS, MASS_ABS, MASS_REL, Buffers, assert_close_bf16,
+                           check_topk, config, f64, ring_to_window, run_fwd, run_select,
+                           window_to_ring)
+
+pytestmark = pytest.mark.gpu
+
+# Small workloads that still span several tiles and ragged edge blocks.
+RAGGED = Workload("ragged", B=2, H=2, D=128, frame_h=12, frame_w=20,
+                  local_cache_size=3 * 240, persistent_cache_size=2 * 240,
+                  total_cache_size=5 * 240, max_seq_len=16 * 240, q_frames=2,
+                  topk_ratio=0.25, bias_fraction=0.1, seed=5)
+RAGGED64 = dataclasses.replace(RAGGED, name="ragged64", D=64, seed=6, frame_h=20, frame_w=12,
+                               local_cache_size=4 * 240, total_cache_size=6 * 240, q_frames=1)
+ODDQB = Workload("oddqb", B=1, H=3, D=128, frame_h=16, frame_w=24,
+                 local_cache_size=2 * 384, persistent_cache_size=384, total_cache_size=3 * 384,
+                 max_seq_len=8 * 384, q_frames=1, topk_ratio=0.5, seed=7)
+
+
+def _mass_to_phys(ml_logical, ring_head, local_frames, W, nbf):
+    B, H, _ = ml_logical.shape
+    out = np.zeros((B, H, W * nbf))
+    for lid in range(local_frames * nbf):
+        phys = ((ring_head + lid // nbf) % W) * nbf + lid % nbf
+        out[:, :, phys] = ml_logical[:, :, lid]
+    return out
+
+
+def _run_case(wl, dev, ring_head=0, local_frames=None, persistent_filled=True, cfg_over=None,
+              qblocks=None, heads=None, check_mass=True):
+    cfg = config(wl, **(cfg_over or {}))
+    inp = decode_inputs(wl, persistent_filled=persistent_filled)
+    W, tf = wl.window_frames, wl.tokens_per_frame
+    lf = W if local_frames is None else local_frames
+    # place the first lf window frames of the generated ring at ring_head
+    win = inp["k_local"][:, :lf * tf]
+    vin = inp["v_local"][:, :lf * tf]
+    kring = window_to_ring(win, ring_head, W, tf)
+    vring = window_to_ring(vin, ring_head, W, tf)
+    d = {k: v.to(dev) for k, v in inp.items()}
+    kring, vring = kring.to(dev), vring.to(dev)
+    buf = Buffers(cfg, wl, wl.q_frames, lf, dev)
+    run_select(buf, d["q"], wl.q_frames, kring, lf, ring_head)
+    run_fwd(buf, d["q"], wl.q_frames, d["k_pers"], d["v_pers"], d["pers_len"], kring, vring,
+            lf, ring_head, mass=check_mass)
+    torch.cuda.synchronize()
+    assert int(buf.status.item()) == 0
+
+    # --- selection
+    kwin = ring_to_window(kring.cpu(), ring_head, lf, W, tf)
+    vwin = ring_to_window(vring.cpu(), ring_head, lf, W, tf)
+    idx_o, sc_o = orc.select_blocks(f64(inp["q"]), f64(kwin), wl.frame_h, wl.frame_w,
+                                    wl.topk_ratio, use_sparse=bool(cfg.use_local_block_sparse_attn))
+    k = buf.k
+    assert idx_o.shape[-1] == k
+    assert np.allclose(buf.scores.cpu().numpy(), sc_o, rtol=0, atol=1e-5)
+    idx_g = buf.idx.cpu().numpy()
+    frac = check_topk(idx_g, buf.cnt.cpu().numpy(), sc_o, k)
+
+    # --- forward, on the GPU's selection
+    O, lse, mp, ml = orc.attn_fwd(f64(inp["q"]), f64(inp["k_pers"]), f64(inp["v_pers"]),
+                                  inp["pers_len"].numpy(), f64(kwin), f64(vwin), idx_g[..., :k],
+                                  wl.frame_h, wl.frame_w, heads=heads, qblocks=qblocks)
+    out = f64(buf.out)
+    lse_g = buf.lse.cpu().numpy()
+    sel = ~np.isnan(lse)
+    assert sel.any()
+    rows = ~np.isnan(O[..., 0, 0]) if heads is None else None
+    if heads is None and qblocks is None:
+        assert_close_bf16(out, O, wl.name + " out")
+        assert np.abs(lse_g - lse).max() <= LSE_ABS
+    else:
+        for b, h in heads:
+            m = sel[b, h]
+            assert_close_bf16(out[b, m, h], O[b, m, h], f"{wl.name} out b{b}h{h}")
+            assert np.abs(lse_g[b, h, m] - lse[b, h, m]).max() <= LSE_ABS
+    if check_mass:
+        mlg = buf.mass_local.cpu().numpy()
+        mpg = buf.mass_pers.cpu().numpy()
+        # every query row's probabilities sum to one
+        tot = mlg.sum(-1) + mpg.sum(-1)
+        assert np.allclose(tot, wl.nq, rtol=1e-4), tot
+        if heads is None and qblocks is None:
+            want_l = _mass_to_phys(ml, ring_head, lf, W, buf.nbf)
+            assert np.allclose(mlg, want_l, rtol=MASS_REL, atol=MASS_ABS)
+            assert np.allclose(mpg, mp, rtol=MASS_REL, atol=MASS_ABS)
+    return frac
+
+
+def test_wait_selftest_times_out_and_reports(cuda_dev):
+    st = torch.zeros(1, dtype=torch.int32, device=cuda_dev)
+    P.pbsa_wait_selftest(st, 20_000_000)
+    torch.cuda.synchronize()
+    assert int(st.item()) == P.PBSA_ERR_TIMEOUT
+    # the context is still usable
+    x = torch.ones(4, device=cuda_dev)
+    assert float(x.sum().item()) == 4.0
+
+
+def test_tiny(cuda_dev):
+    _run_case(WORKLOADS["tiny"], cuda_dev)
+
+
+@pytest.mark.parametrize("ring_head", [0, 2])
+def test_ragged_blocks_and_ring(cuda_dev, ring_head):
+    _run_case(RAGGED, cuda_dev, ring_head=ring_head)
+
+
+def test_ragged_d64_partial_window(cuda_dev):
+    _run_case(RAGGED64, cuda_dev, ring_head=3, local_frames=2)
+
+
+def test_empty_persistent_cache(cuda_dev):
+    _run_case(RAGGED, cuda_dev, persistent_filled=False)
+
+
+def test_odd_query_block_count(cuda_dev):
+    _run_case(ODDQB, cuda_dev, ring_head=1)
+
+
+def test_dense_local_window_flag_off(cuda_dev):
+    _run_case(RAGGED, cuda_dev, cfg_over=dict(use_local_block_sparse_attn=False))
+
+
+def test_forward_without_mass(cuda_dev):
+    _run_case(RAGGED, cuda_dev, check_mass=False)
+
+
+def test_decode_full_size_sampled(cuda_dev):
+    """The page-sized decode step (H=12, D=128, 30x52 frames, 168 + 168 blocks, k=21), in
+    the launch configuration the benchmark times; the oracle recomputes sampled query
+    blocks (ragged ones included) of sampled heads, the selection of every query block,
+    and the masses through the probability-sum invariant."""
+    wl = WORKLOADS["decode"]
+    frac = _run_case(wl, cuda_dev, qblocks=[0, 6, 20, 27, 41, 55, 83], heads=[(0, 0), (0, 7), (0, 11)])
+    print(f"decode: exact top-k fraction {frac:.3f}")
+
+
+def test_decode_full_size_one_head_mass(cuda_dev):
+    wl = dataclasses.replace(WORKLOADS["decode"], H=1)
+    _run_case(wl, cuda_dev)
