@@ -1,8 +1,854 @@
-// attn_bwd.cu - PBSA backward (placeholder until the kernel lands).
+// attn_bwd.cu - PBSA backward on sm_100a (TMA + tcgen05 + TMEM).
+//
+// Sparse Forcing project page (kernel features): full gradient support for training.
+// Gradients of sum(O * dO) with the block selection held fixed:
+//   P  = exp(S - lse) with S = Q K^T / sqrt(D)   (recomputed from the forward's lse)
+//   dV = P^T dO,   dP = dO V^T,   Delta = rowsum(dO * O),   dS = P * (dP - Delta)
+//   dQ = dS K / sqrt(D),   dK = dS^T Q / sqrt(D)
+// Deterministic, no atomics, three kernels:
+//  1. delta_kernel: Delta per query row (one pass over O and dO).
+//  2. dkdv_kernel: one CTA per key tile (128 keys: 16 compacted 8-row groups of the
+//     persistent slots, or a pair of local blocks); it loops over the query tiles that
+//     attend to those keys (all of them for persistent keys; for local blocks the query
+//     tiles whose query blocks selected either block).  S^T = K Q^T and dP^T = V dO^T land
+//     in TMEM (lanes = keys); each thread owns one key row, forms P^T and dS^T, writes them
+//     as bf16 back over S^T / dP^T, and two TS MMAs accumulate dV += P^T dO and
+//     dK += dS^T Q in TMEM (dO and Q tiles read MN-major from shared memory).
+//  3. dq_kernel: one CTA per query tile (the forward's tiling); per key tile S = Q K^T and
+//     dP = dO V^T in TMEM, each thread (one query row) forms dS, writes it as bf16 over S,
+//     and a TS MMA accumulates dQ += dS K (K read MN-major).
+// Warp roles in 2 and 3: warps 0-3 one row per thread, warp 4 TMA producer, warp 5 MMA.
+#include <cuda_bf16.h>
+#include <math_constants.h>
+
+#include "pbsa_device.cuh"
 #include "pbsa_internal.cuh"
 
 namespace pbsa {
 
-cudaError_t launch_attn_bwd(const BwdArgs&, cudaStream_t) { return cudaErrorNotSupported; }
+namespace {
+
+constexpr uint32_t kHalf = 128 * 128;   // 128 rows x 64 bf16 channels
+constexpr int kThreads = 192;
+constexpr int kNst = 2;
+constexpr float kLog2e = 1.4426950408889634f;
+
+
+// ----------------------------------------------------------------------- delta
+__global__ void __launch_bounds__(256) delta_kernel(const __nv_bfloat16* __restrict__ o,
+                                                    const __nv_bfloat16* __restrict__ d_o,
+                                                    float* __restrict__ delta, int nq, int H,
+                                                    int D, long long nrows) {
+    // one row (token, head) per 16 threads, 8 channels per thread per step
+    const long long row = (long long)blockIdx.x * 16 + threadIdx.x / 16;
+    const int sub = threadIdx.x % 16;
+    float acc = 0.f;
+    if (row < nrows) {
+        const __nv_bfloat16* a = o + row * D;
+        const __nv_bfloat16* b = d_o + row * D;
+        for (int c = sub * 8; c < D; c += 128) {
+            const uint4 va = __ldg(reinterpret_cast<const uint4*>(a + c));
+            const uint4 vb = __ldg(reinterpret_cast<const uint4*>(b + c));
+            const __nv_bfloat162* pa = reinterpret_cast<const __nv_bfloat162*>(&va);
+            const __nv_bfloat162* pb = reinterpret_cast<const __nv_bfloat162*>(&vb);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 fa = __bfloat1622float2(pa[e]);
+                const float2 fb = __bfloat1622float2(pb[e]);
+                acc = fmaf(fa.x, fb.x, acc);
+                acc = fmaf(fa.y, fb.y, acc);
+            }
+        }
+    }
+#pragma unroll
+    for (int off = 8; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off, 16);
+    if (row < nrows && sub == 0) {
+        // row = (b * nq + t) * H + h  ->  delta[(b * H + h) * nq + t]
+        const long long bt = row / H;
+        const int h = (int)(row % H);
+        const long long b = bt / nq, t = bt % nq;
+        delta[(b * H + h) * nq + t] = acc;
+    }
+}
+
+// --------------------------------------------------------- persistent group table
+// Builds, with one warp, the compacted list of the occupied slots' 8-row groups: row
+// index of each group in the [B*H*S*64, D] slot store.  Returns the group count.
+__device__ int build_groups(const int32_t* pers_len, int bh, int S, int32_t* grp_row,
+                            int32_t* status) {
+    const int lane = threadIdx.x & 31;
+    int run = 0;
+    for (int s0 = 0; s0 < S; s0 += 32) {
+        const int s = s0 + lane;
+        int len = (s < S) ? pers_len[(size_t)bh * S + s] : 0;
+        if (len < 0 || len > 64 || (len & 7)) {
+            set_status(status, PBSA_ERR_DEVICE_CHECK);
+            len = 0;
+        }
+        const int ng = len >> 3;
+        int inc = ng;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, inc, o);
+            if (lane >= o) inc += v;
+        }
+        const int gstart = run + inc - ng;
+        for (int i = 0; i < ng; ++i) grp_row[gstart + i] = ((bh * S) + s) * 64 + 8 * i;
+        run += __shfl_sync(0xffffffffu, inc, 31);
+    }
+    return run;
+}
+
+constexpr int B_COUNT = 12;  // mbarrier slots reserved per CTA
+
+// ===================================================================== dK / dV
+struct DkdvPlan {
+    uint32_t k, v, q, dq_o, lse, dl, grp_row, qtl, qsel, bars, misc, total;
+};
+
+__host__ __device__ inline DkdvPlan dkdv_plan(int D, int S, int n_qt) {
+    DkdvPlan p;
+    const uint32_t nh = D / 64;
+    p.k = 0;
+    p.v = p.k + nh * kHalf;
+    p.q = p.v + nh * kHalf;                 // kNst stages of Q
+    p.dq_o = p.q + kNst * nh * kHalf;       // kNst stages of dO
+    p.lse = p.dq_o + kNst * nh * kHalf;     // kNst x 128 fp32 (log2 units, +inf = padding)
+    p.dl = p.lse + kNst * 128 * 4;          // kNst x 128 fp32 Delta
+    p.grp_row = p.dl + kNst * 128 * 4;      // 8*S
+    p.qtl = p.grp_row + 4u * 8u * S;        // query tile list
+    p.qsel = p.qtl + 4u * n_qt;             // 4 selection bits per listed query tile
+    p.bars = (p.qsel + 4u * n_qt + 7u) & ~7u;
+    p.misc = p.bars + 8u * B_COUNT;
+    p.total = p.misc + 4u * 8u;
+    return p;
+}
+
+struct DkdvKernelArgs {
+    BwdArgs a;
+    int n_pt_max;  // persistent key tiles per (b, h) in the grid
+    int n_qt;      // query tiles per (b, h)
+};
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1) dkdv_kernel(const __grid_constant__ DkdvKernelArgs ka) {
+    constexpr int NH = D / 64;
+    constexpr uint32_t TILE = NH * kHalf;
+    constexpr uint32_t kTmS = 0, kTmP = 128, kTmDV = 256, kTmDK = 256 + D;
+    const BwdArgs& a = ka.a;
+    const Geo& g = a.g;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+    const int S = g.S;
+    const DkdvPlan PL = dkdv_plan(D, S, ka.n_qt);
+    uint8_t* sK = sm + PL.k;
+    uint8_t* sV = sm + PL.v;
+    uint8_t* sQ = sm + PL.q;
+    uint8_t* sDO = sm + PL.dq_o;
+    float* s_lse = reinterpret_cast<float*>(sm + PL.lse);
+    float* s_dl = reinterpret_cast<float*>(sm + PL.dl);
+    int32_t* grp_row = reinterpret_cast<int32_t*>(sm + PL.grp_row);
+    int32_t* qtl = reinterpret_cast<int32_t*>(sm + PL.qtl);
+    int32_t* qsel = reinterpret_cast<int32_t*>(sm + PL.qsel);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + PL.bars);
+    int* misc = reinterpret_cast<int*>(sm + PL.misc);
+    volatile int* abort_flag = misc + 1;
+
+    const int h = blockIdx.y, b = blockIdx.z, bh = b * g.H + h;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int qb_total = a.q_frames * g.nbf;
+    const int nq = a.q_frames * g.tf;
+    const int nl = a.local_frames * g.nbf;
+    const bool pers_tile = (int)blockIdx.x < ka.n_pt_max;
+    const int tile = pers_tile ? blockIdx.x : blockIdx.x - ka.n_pt_max;
+
+    uint64_t* kv_full = &bars[0];      // K and V tiles of this CTA (once)
+    uint64_t* qd_full = &bars[1];      // [kNst] Q + dO + lse/Delta of a query tile
+    uint64_t* qd_empty = &bars[3];     // [kNst]
+    uint64_t* sdp_full = &bars[5];     // S^T and dP^T ready
+    uint64_t* pds_full = &bars[6];     // P^T and dS^T written (128 arrivals)
+    uint64_t* pass_done = &bars[7];    // dV/dK MMAs of a query tile done
+    uint64_t* drain = &bars[8];
+    if (threadIdx.x == 0) {
+        mbar_init(kv_full, 1);
+        for (int s = 0; s < kNst; ++s) {
+            mbar_init(&qd_full[s], 1 + 32);  // producer expect_tx + 32 lse/Delta loaders
+            mbar_init(&qd_empty[s], 1);
+        }
+        mbar_init(sdp_full, 1);
+        mbar_init(pds_full, 128);
+        mbar_init(pass_done, 1);
+        mbar_init(drain, 1);
+        misc[1] = 0;
+        fence_barrier_init();
+    }
+    if (warp == 5) tmem_alloc(reinterpret_cast<uint32_t*>(misc + 0), 512);
+
+    // key set of this CTA
+    int G = 0, L0 = -1, L1 = -1;
+    if (pers_tile) {
+        if (warp == 0) {
+            G = build_groups(a.pers_len, bh, S, grp_row, a.status);
+            if (lane == 0) misc[2] = G;
+        }
+    } else {
+        L0 = 2 * tile;
+        L1 = (2 * tile + 1 < nl) ? 2 * tile + 1 : -1;
+    }
+    __syncthreads();
+    if (pers_tile) G = misc[2];
+    // the query tiles that see these keys, with selection bits
+    //   bit (2*kb + hq): key block kb (0/1) was selected by query block 2*qt + hq
+    if (warp < 4) {
+        const int n_qt = ka.n_qt;
+        int count = 0;
+        for (int t0 = 0; t0 < n_qt; t0 += 128) {
+            const int qt = t0 + threadIdx.x;
+            int bits = 0;
+            if (qt < n_qt) {
+                if (pers_tile) {
+                    bits = 0xF;
+                } else {
+                    for (int hq = 0; hq < 2; ++hq) {
+                        const int qb = 2 * qt + hq;
+                        if (qb >= qb_total) continue;
+                        const int c = min(max(a.cnt[(size_t)bh * qb_total + qb], 0), a.idx_stride);
+                        const int32_t* row = a.idx + ((size_t)bh * qb_total + qb) * a.idx_stride;
+                        for (int i = 0; i < c; ++i) {
+                            const int v = row[i];
+                            if (v == L0) bits |= 1 << (0 + hq);
+                            if (L1 >= 0 && v == L1) bits |= 1 << (2 + hq);
+                        }
+                    }
+                }
+            }
+            // block-wide compaction of the tiles with bits != 0 (4 warps)
+            const unsigned m = __ballot_sync(0xffffffffu, bits != 0);
+            __shared__ int wcount[4];
+            if (lane == 0) wcount[warp] = __popc(m);
+            named_bar_sync(1, 128);
+            int base = count;
+            for (int w = 0; w < warp; ++w) base += wcount[w];
+            if (bits) {
+                const int pos = base + __popc(m & ((1u << lane) - 1u));
+                qtl[pos] = qt;
+                qsel[pos] = bits;
+            }
+            count += wcount[0] + wcount[1] + wcount[2] + wcount[3];
+            named_bar_sync(1, 128);
+        }
+        if (threadIdx.x == 0) misc[3] = count;
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = static_cast<uint32_t>(misc[0]);
+    const int n_items = misc[3];
+    const bool live = pers_tile ? (tile * 16 < G) : true;
+
+    if (live && warp == 4) {
+        // ---------------------------------------------------------- producer
+        if (lane == 0) {
+            mbar_arrive_expect_tx(kv_full, 2 * TILE);
+            if (pers_tile) {
+                for (int c = 0; c < 16; ++c) {
+                    const int row = grp_row[min(tile * 16 + c, G - 1)];
+                    for (int hh = 0; hh < NH; ++hh) {
+                        tma_load_2d(sK + hh * kHalf + c * 1024, &a.tm_kp, kv_full, hh * 64, row);
+                        tma_load_2d(sV + hh * kHalf + c * 1024, &a.tm_vp, kv_full, hh * 64, row);
+                    }
+                }
+            } else {
+                for (int kb = 0; kb < 2; ++kb) {
+                    const int L = (kb == 1 && L1 >= 0) ? L1 : L0;
+                    const int pos = L / g.nbf, i = L % g.nbf;
+                    const int fr = b * g.W + (a.ring_head + pos) % g.W;
+                    for (int hh = 0; hh < NH; ++hh) {
+                        tma_load_5d(sK + hh * kHalf + kb * (kHalf / 2), &a.tm_kl, kv_full, hh * 64, h,
+                                    8 * (i % g.nbx), 8 * (i / g.nbx), fr);
+                        tma_load_5d(sV + hh * kHalf + kb * (kHalf / 2), &a.tm_vl, kv_full, hh * 64, h,
+                                    8 * (i % g.nbx), 8 * (i / g.nbx), fr);
+                    }
+                }
+            }
+        }
+        __syncwarp();
+        int issued = 0;
+        for (int j = 0; j < n_items; ++j) {
+            const int st = j % kNst;
+            if (j >= kNst) {
+                const bool w = __all_sync(0xffffffffu, mbar_wait(&qd_empty[st], ((j / kNst) - 1) & 1, abort_flag, a.status));
+                if (!w) break;
+            }
+            const int qt = qtl[j];
+            if (lane == 0) {
+                mbar_arrive_expect_tx(&qd_full[st], 2 * TILE);
+                for (int hq = 0; hq < 2; ++hq) {
+                    const int qb = min(2 * qt + hq, qb_total - 1);
+                    const int f = qb / g.nbf, i = qb % g.nbf;
+                    for (int hh = 0; hh < NH; ++hh) {
+                        tma_load_5d(sQ + st * TILE + hh * kHalf + hq * (kHalf / 2), &a.tm_q, &qd_full[st],
+                                    hh * 64, h, 8 * (i % g.nbx), 8 * (i / g.nbx), b * a.q_frames + f);
+                        tma_load_5d(sDO + st * TILE + hh * kHalf + hq * (kHalf / 2), &a.tm_do, &qd_full[st],
+                                    hh * 64, h, 8 * (i % g.nbx), 8 * (i / g.nbx), b * a.q_frames + f);
+                    }
+                }
+            }
+            // lse (log2 units) and Delta of the tile's 128 query rows; +inf lse masks padding
+            for (int r = lane; r < 128; r += 32) {
+                const int hq = r >> 6, qb = 2 * qt + hq, rr = r & 63;
+                float l2 = CUDART_INF_F, dl = 0.f;
+                if (qb < qb_total) {
+                    const int f = qb / g.nbf, i = qb % g.nbf;
+                    const int y = 8 * (i / g.nbx) + (rr >> 3), x = 8 * (i % g.nbx) + (rr & 7);
+                    if (y < g.fh && x < g.fw) {
+                        const size_t t = (size_t)bh * nq + f * g.tf + y * g.fw + x;
+                        l2 = a.lse[t] * kLog2e;
+                        dl = a.delta[t];
+                    }
+                }
+                s_lse[st * 128 + r] = l2;
+                s_dl[st * 128 + r] = dl;
+            }
+            mbar_arrive(&qd_full[st]);
+            ++issued;
+        }
+        if (lane == 0 && *abort_flag) {
+            mbar_wait_drain(kv_full, 0, 100000000ull);
+            for (int j = max(0, issued - kNst); j < issued; ++j)
+                mbar_wait_drain(&qd_full[j % kNst], (j / kNst) & 1, 100000000ull);
+        }
+    } else if (live && warp == 5) {
+        // ---------------------------------------------------------------- MMA
+        if (lane == 0) {
+            constexpr uint32_t id_s = idesc_bf16(128, 128, false, false);
+            constexpr uint32_t id_g = idesc_bf16(128, D, false, true);
+            bool ok = mbar_wait(kv_full, 0, abort_flag, a.status);
+            const uint32_t kb = smem_u32(sK), vb = smem_u32(sV);
+            for (int j = 0; ok && j < n_items; ++j) {
+                const int st = j % kNst;
+                if (!mbar_wait(&qd_full[st], (j / kNst) & 1, abort_flag, a.status)) { ok = false; break; }
+                if (j > 0 && !mbar_wait(pass_done, (j - 1) & 1, abort_flag, a.status)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t qb_ = smem_u32(sQ + st * TILE), ob = smem_u32(sDO + st * TILE);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
+                    umma_ss(tmem + kTmS, sdesc_sw128(kb + off, 16, 1024), sdesc_sw128(qb_ + off, 16, 1024), id_s, kk > 0);
+                }
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
+                    umma_ss(tmem + kTmP, sdesc_sw128(vb + off, 16, 1024), sdesc_sw128(ob + off, 16, 1024), id_s, kk > 0);
+                }
+                umma_commit(sdp_full);
+                if (!mbar_wait(pds_full, j & 1, abort_flag, a.status)) { ok = false; break; }
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    umma_ts(tmem + kTmDV, tmem + kTmS + kk * 8, sdesc_sw128(ob + kk * 2048, kHalf, 1024), id_g,
+                            (j > 0 || kk > 0) ? 1u : 0u);
+                }
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    umma_ts(tmem + kTmDK, tmem + kTmP + kk * 8, sdesc_sw128(qb_ + kk * 2048, kHalf, 1024), id_g,
+                            (j > 0 || kk > 0) ? 1u : 0u);
+                }
+                umma_commit(pass_done);
+                umma_commit(&qd_empty[st]);
+            }
+            if (!ok) {
+                umma_commit(drain);
+                mbar_wait_drain(drain, 0, 100000000ull);
+            }
+        }
+    } else if (live) {
+        // ------------------------------------------------- key-row threads (warps 0-3)
+        const int r = threadIdx.x;
+        const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+        const float sl2 = kLog2e / sqrtf(static_cast<float>(D));
+        bool key_valid;
+        int kbr = 0;
+        if (pers_tile) {
+            key_valid = tile * 16 + (r >> 3) < G;
+        } else {
+            kbr = r >> 6;
+            const int L = kbr ? L1 : L0;
+            if (L < 0) {
+                key_valid = false;
+            } else {
+                const int i = L % g.nbf, rr = r & 63;
+                key_valid = (8 * (i / g.nbx) + (rr >> 3) < g.fh) && (8 * (i % g.nbx) + (rr & 7) < g.fw);
+            }
+        }
+        auto wwait = [&](uint64_t* bar, uint32_t parity) -> bool {
+            return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, a.status));
+        };
+        bool ok = true;
+        for (int j = 0; j < n_items; ++j) {
+            const int st = j % kNst;
+            // lse/Delta of this query tile (written by the producer warp)
+            if (!wwait(&qd_full[st], (j / kNst) & 1)) { ok = false; break; }
+            if (!wwait(sdp_full, j & 1)) { ok = false; break; }
+            tc_fence_after();
+            const int bits = qsel[j];
+            const bool sel0 = key_valid && ((bits >> (2 * kbr + 0)) & 1);
+            const bool sel1 = key_valid && ((bits >> (2 * kbr + 1)) & 1);
+            const float* lse2 = s_lse + st * 128;
+            const float* dl = s_dl + st * 128;
+            uint32_t pk[32], dk[32];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                uint32_t sv[32], pv[32];
+                tmem_ld32(tmem + lane_base + kTmS + 32 * c, sv);
+                tmem_ld32(tmem + lane_base + kTmP + 32 * c, pv);
+                tmem_ld_wait();
+                const bool sel = c < 2 ? sel0 : sel1;
+#pragma unroll
+                for (int e = 0; e < 32; e += 2) {
+                    const int q = 32 * c + e;
+                    float p0 = sel ? fast_exp2(__uint_as_float(sv[e]) * sl2 - lse2[q]) : 0.f;
+                    float p1 = sel ? fast_exp2(__uint_as_float(sv[e + 1]) * sl2 - lse2[q + 1]) : 0.f;
+                    const float d0 = p0 * (__uint_as_float(pv[e]) - dl[q]);
+                    const float d1 = p1 * (__uint_as_float(pv[e + 1]) - dl[q + 1]);
+                    pk[16 * (c & 1) + e / 2] = pack_bf16x2(p0, p1);
+                    dk[16 * (c & 1) + e / 2] = pack_bf16x2(d0, d1);
+                }
+                if (c & 1) {
+                    tmem_st32(tmem + lane_base + kTmS + 32 * (c >> 1), pk);
+                    tmem_st32(tmem + lane_base + kTmP + 32 * (c >> 1), dk);
+                }
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(pds_full);
+        }
+        ok = named_bar_and(1, 128, ok);
+        if (ok && n_items > 0) {
+            ok = named_bar_and(1, 128, wwait(pass_done, (n_items - 1) & 1));
+            tc_fence_after();
+        }
+        if (ok) {
+            // destination row of this key
+            float* dk_row = nullptr;
+            float* dv_row = nullptr;
+            if (key_valid) {
+                if (pers_tile) {
+                    const size_t row = (size_t)grp_row[tile * 16 + (r >> 3)] + (r & 7);
+                    dk_row = a.dk_pers + row * D;
+                    dv_row = a.dv_pers + row * D;
+                } else {
+                    const int L = kbr ? L1 : L0;
+                    const int pos = L / g.nbf, i = L % g.nbf, rr = r & 63;
+                    const int phys = (a.ring_head + pos) % g.W;
+                    const int y = 8 * (i / g.nbx) + (rr >> 3), x = 8 * (i % g.nbx) + (rr & 7);
+                    const size_t tok = ((size_t)b * g.W + phys) * g.tf + y * g.fw + x;
+                    dk_row = a.dk_local + (tok * g.H + h) * D;
+                    dv_row = a.dv_local + (tok * g.H + h) * D;
+                }
+            }
+            const float isd = 1.0f / sqrtf(static_cast<float>(D));
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t v[32], w[32];
+                if (n_items > 0) {
+                    tmem_ld32(tmem + lane_base + kTmDV + 32 * c, v);
+                    tmem_ld32(tmem + lane_base + kTmDK + 32 * c, w);
+                    tmem_ld_wait();
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) v[e] = w[e] = 0u;
+                }
+                if (key_valid) {
+#pragma unroll
+                    for (int e = 0; e < 32; e += 4) {
+                        *reinterpret_cast<float4*>(dv_row + 32 * c + e) =
+                            make_float4(__uint_as_float(v[e]), __uint_as_float(v[e + 1]),
+                                        __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
+                        *reinterpret_cast<float4*>(dk_row + 32 * c + e) =
+                            make_float4(__uint_as_float(w[e]) * isd, __uint_as_float(w[e + 1]) * isd,
+                                        __uint_as_float(w[e + 2]) * isd, __uint_as_float(w[e + 3]) * isd);
+                    }
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 5) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// ========================================================================== dQ
+struct DqPlan {
+    uint32_t q, dq_o, k, v, grp_row, uni_blk, uni_bits, bars, misc, total;
+};
+
+__host__ __device__ inline DqPlan dq_plan(int D, int S, int ucap) {
+    DqPlan p;
+    const uint32_t nh = D / 64;
+    p.q = 0;
+    p.dq_o = p.q + nh * kHalf;
+    p.k = p.dq_o + nh * kHalf;
+    p.v = p.k + kNst * nh * kHalf;
+    p.grp_row = p.v + kNst * nh * kHalf;
+    p.uni_blk = p.grp_row + 4u * 8u * S;
+    p.uni_bits = p.uni_blk + 4u * ucap;
+    p.bars = (p.uni_bits + 4u * ucap + 7u) & ~7u;
+    p.misc = p.bars + 8u * 16u;
+    p.total = p.misc + 4u * 8u;
+    return p;
+}
+
+struct DqKernelArgs {
+    BwdArgs a;
+    int ucap;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__ DqKernelArgs ka) {
+    constexpr int NH = D / 64;
+    constexpr uint32_t TILE = NH * kHalf;
+    constexpr uint32_t kTmS = 0, kTmP = 128, kTmQ = 256;
+    const BwdArgs& a = ka.a;
+    const Geo& g = a.g;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+    const int S = g.S;
+    const int ucap = ka.ucap;
+    const DqPlan PL = dq_plan(D, S, ucap);
+    uint8_t* sQ = sm + PL.q;
+    uint8_t* sDO = sm + PL.dq_o;
+    uint8_t* sK = sm + PL.k;
+    uint8_t* sV = sm + PL.v;
+    int32_t* grp_row = reinterpret_cast<int32_t*>(sm + PL.grp_row);
+    int32_t* uni_blk = reinterpret_cast<int32_t*>(sm + PL.uni_blk);
+    int32_t* uni_bits = reinterpret_cast<int32_t*>(sm + PL.uni_bits);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + PL.bars);
+    int* misc = reinterpret_cast<int*>(sm + PL.misc);
+    volatile int* abort_flag = misc + 1;
+    uint64_t* q_full = &bars[0];
+    uint64_t* k_full = &bars[1];    // [kNst]
+    uint64_t* v_full = &bars[3];    // [kNst]
+    uint64_t* kv_empty = &bars[5];  // [kNst]
+    uint64_t* sdp_full = &bars[7];
+    uint64_t* ds_full = &bars[8];
+    uint64_t* dq_done = &bars[9];
+    uint64_t* drain = &bars[10];
+
+    const int tile = blockIdx.x, h = blockIdx.y, b = blockIdx.z, bh = b * g.H + h;
+    const int qb_total = a.q_frames * g.nbf;
+    const int nq = a.q_frames * g.tf;
+    const int qb0 = 2 * tile;
+    const int qb1 = (2 * tile + 1 < qb_total) ? 2 * tile + 1 : -1;
+    const int nl = a.local_frames * g.nbf;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        mbar_init(q_full, 1);
+        for (int s = 0; s < kNst; ++s) {
+            mbar_init(&k_full[s], 1);
+            mbar_init(&v_full[s], 1);
+            mbar_init(&kv_empty[s], 1);
+        }
+        mbar_init(sdp_full, 1);
+        mbar_init(ds_full, 128);
+        mbar_init(dq_done, 1);
+        mbar_init(drain, 1);
+        misc[1] = 0;
+        fence_barrier_init();
+    }
+    if (warp == 5) tmem_alloc(reinterpret_cast<uint32_t*>(misc + 0), 512);
+    if (warp == 0) {
+        const int G = build_groups(a.pers_len, bh, S, grp_row, a.status);
+        if (lane == 0) misc[2] = G;
+    }
+    if (warp == 1 && lane == 0) {
+        const int c0 = min(max(a.cnt[(size_t)bh * qb_total + qb0], 0), a.idx_stride);
+        const int c1 = qb1 >= 0 ? min(max(a.cnt[(size_t)bh * qb_total + qb1], 0), a.idx_stride) : 0;
+        const int32_t* i0 = a.idx + ((size_t)bh * qb_total + qb0) * a.idx_stride;
+        const int32_t* i1 = a.idx + ((size_t)bh * qb_total + (qb1 >= 0 ? qb1 : qb0)) * a.idx_stride;
+        int p = 0, q = 0, u = 0;
+        while (p < c0 || q < c1) {
+            if (u == ucap) {
+                set_status(a.status, PBSA_ERR_DEVICE_CHECK);
+                break;
+            }
+            const int v0 = p < c0 ? i0[p] : 0x7fffffff;
+            const int v1 = q < c1 ? i1[q] : 0x7fffffff;
+            int blk, bits;
+            if (v0 == v1) {
+                blk = v0; bits = 3; ++p; ++q;
+            } else if (v0 < v1) {
+                blk = v0; bits = 1; ++p;
+            } else {
+                blk = v1; bits = 2; ++q;
+            }
+            if (blk < 0 || blk >= nl) {
+                set_status(a.status, PBSA_ERR_DEVICE_CHECK);
+                continue;
+            }
+            uni_blk[u] = blk;
+            uni_bits[u] = bits;
+            ++u;
+        }
+        misc[3] = u;
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = static_cast<uint32_t>(misc[0]);
+    const int G = misc[2], U = misc[3];
+    const int n_pt = (G + 15) / 16;
+    const int n_tiles = n_pt + (U + 1) / 2;
+
+    if (warp == 4) {
+        if (lane == 0) {
+            mbar_arrive_expect_tx(q_full, 2 * TILE);
+            for (int hb = 0; hb < 2; ++hb) {
+                const int qb = (hb == 1 && qb1 >= 0) ? qb1 : qb0;
+                const int f = qb / g.nbf, i = qb % g.nbf;
+                for (int hh = 0; hh < NH; ++hh) {
+                    tma_load_5d(sQ + hh * kHalf + hb * (kHalf / 2), &a.tm_q, q_full, hh * 64, h,
+                                8 * (i % g.nbx), 8 * (i / g.nbx), b * a.q_frames + f);
+                    tma_load_5d(sDO + hh * kHalf + hb * (kHalf / 2), &a.tm_do, q_full, hh * 64, h,
+                                8 * (i % g.nbx), 8 * (i / g.nbx), b * a.q_frames + f);
+                }
+            }
+            int issued = 0;
+            for (int it = 0; it < n_tiles; ++it) {
+                const int st = it % kNst;
+                if (it >= kNst && !mbar_wait(&kv_empty[st], ((it / kNst) - 1) & 1, abort_flag, a.status)) break;
+                uint8_t* dk = sK + st * TILE;
+                uint8_t* dv = sV + st * TILE;
+                mbar_arrive_expect_tx(&k_full[st], TILE);
+                mbar_arrive_expect_tx(&v_full[st], TILE);
+                if (it < n_pt) {
+                    for (int c = 0; c < 16; ++c) {
+                        const int row = grp_row[min(it * 16 + c, G - 1)];
+                        for (int hh = 0; hh < NH; ++hh) {
+                            tma_load_2d(dk + hh * kHalf + c * 1024, &a.tm_kp, &k_full[st], hh * 64, row);
+                            tma_load_2d(dv + hh * kHalf + c * 1024, &a.tm_vp, &v_full[st], hh * 64, row);
+                        }
+                    }
+                } else {
+                    const int j = it - n_pt;
+                    for (int hb = 0; hb < 2; ++hb) {
+                        const int L = uni_blk[min(2 * j + hb, U - 1)];
+                        const int pos = L / g.nbf, i = L % g.nbf;
+                        const int fr = b * g.W + (a.ring_head + pos) % g.W;
+                        for (int hh = 0; hh < NH; ++hh) {
+                            tma_load_5d(dk + hh * kHalf + hb * (kHalf / 2), &a.tm_kl, &k_full[st], hh * 64, h,
+                                        8 * (i % g.nbx), 8 * (i / g.nbx), fr);
+                            tma_load_5d(dv + hh * kHalf + hb * (kHalf / 2), &a.tm_vl, &v_full[st], hh * 64, h,
+                                        8 * (i % g.nbx), 8 * (i / g.nbx), fr);
+                        }
+                    }
+                }
+                ++issued;
+            }
+            if (*abort_flag) {
+                mbar_wait_drain(q_full, 0, 100000000ull);
+                for (int it = max(0, issued - kNst); it < issued; ++it) {
+                    mbar_wait_drain(&k_full[it % kNst], (it / kNst) & 1, 100000000ull);
+                    mbar_wait_drain(&v_full[it % kNst], (it / kNst) & 1, 100000000ull);
+                }
+            }
+        }
+    } else if (warp == 5) {
+        if (lane == 0) {
+            constexpr uint32_t id_s = idesc_bf16(128, 128, false, false);
+            constexpr uint32_t id_g = idesc_bf16(128, D, false, true);
+            bool ok = mbar_wait(q_full, 0, abort_flag, a.status);
+            const uint32_t qbase = smem_u32(sQ), obase = smem_u32(sDO);
+            for (int it = 0; ok && it < n_tiles; ++it) {
+                const int st = it % kNst;
+                if (!mbar_wait(&k_full[st], (it / kNst) & 1, abort_flag, a.status)) { ok = false; break; }
+                if (!mbar_wait(&v_full[st], (it / kNst) & 1, abort_flag, a.status)) { ok = false; break; }
+                if (it > 0 && !mbar_wait(dq_done, (it - 1) & 1, abort_flag, a.status)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t kb = smem_u32(sK + st * TILE), vb = smem_u32(sV + st * TILE);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
+                    umma_ss(tmem + kTmS, sdesc_sw128(qbase + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024), id_s, kk > 0);
+                }
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
+                    umma_ss(tmem + kTmP, sdesc_sw128(obase + off, 16, 1024), sdesc_sw128(vb + off, 16, 1024), id_s, kk > 0);
+                }
+                umma_commit(sdp_full);
+                if (!mbar_wait(ds_full, it & 1, abort_flag, a.status)) { ok = false; break; }
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    umma_ts(tmem + kTmQ, tmem + kTmS + kk * 8, sdesc_sw128(kb + kk * 2048, kHalf, 1024), id_g,
+                            (it > 0 || kk > 0) ? 1u : 0u);
+                umma_commit(dq_done);
+                umma_commit(&kv_empty[st]);
+            }
+            if (!ok) {
+                umma_commit(drain);
+                mbar_wait_drain(drain, 0, 100000000ull);
+            }
+        }
+    } else {
+        const int r = threadIdx.x;
+        const int hq = r >> 6, rr = r & 63, dy = rr >> 3, dx = rr & 7;
+        const int qbr = hq ? qb1 : qb0;
+        const int qbv = qbr >= 0 ? qbr : qb0;
+        const int qf = qbv / g.nbf, qi = qbv % g.nbf;
+        const int qy = 8 * (qi / g.nbx) + dy, qx = 8 * (qi % g.nbx) + dx;
+        const bool row_valid = qbr >= 0 && qy < g.fh && qx < g.fw;
+        const size_t tok = (size_t)qf * g.tf + qy * g.fw + qx;
+        const float lse2 = row_valid ? a.lse[(size_t)bh * nq + tok] * kLog2e : CUDART_INF_F;
+        const float dl = row_valid ? a.delta[(size_t)bh * nq + tok] : 0.f;
+        const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+        const float sl2 = kLog2e / sqrtf(static_cast<float>(D));
+        auto wwait = [&](uint64_t* bar, uint32_t parity) -> bool {
+            return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, a.status));
+        };
+        bool ok = true;
+        for (int it = 0; it < n_tiles; ++it) {
+            if (!wwait(sdp_full, it & 1)) { ok = false; break; }
+            tc_fence_after();
+            int nvc = 128;
+            bool sel0 = true, sel1 = true;
+            int hv0 = 8, wv0 = 8, hv1 = 8, wv1 = 8;
+            const bool local = it >= n_pt;
+            if (!local) {
+                nvc = min(128, 8 * (G - 16 * it));
+            } else {
+                const int u0 = 2 * (it - n_pt);
+                const bool has1 = u0 + 1 < U;
+                const int L0 = uni_blk[u0], L1 = has1 ? uni_blk[u0 + 1] : L0;
+                sel0 = (uni_bits[u0] >> hq) & 1;
+                sel1 = has1 && ((uni_bits[u0 + 1] >> hq) & 1);
+                const int i0 = L0 % g.nbf, i1 = L1 % g.nbf;
+                hv0 = min(8, g.fh - 8 * (i0 / g.nbx));
+                wv0 = min(8, g.fw - 8 * (i0 % g.nbx));
+                hv1 = min(8, g.fh - 8 * (i1 / g.nbx));
+                wv1 = min(8, g.fw - 8 * (i1 % g.nbx));
+            }
+            uint32_t dk[32];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                uint32_t sv[32], pv[32];
+                tmem_ld32(tmem + lane_base + kTmS + 32 * c, sv);
+                tmem_ld32(tmem + lane_base + kTmP + 32 * c, pv);
+                tmem_ld_wait();
+#pragma unroll
+                for (int e = 0; e < 32; e += 2) {
+                    float dsv[2];
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        const int col = 32 * c + e + u;
+                        bool valid;
+                        if (!local) {
+                            valid = col < nvc;
+                        } else {
+                            const int cc = col & 63;
+                            valid = col < 64 ? (sel0 && (cc >> 3) < hv0 && (cc & 7) < wv0)
+                                             : (sel1 && (cc >> 3) < hv1 && (cc & 7) < wv1);
+                        }
+                        const float p = valid ? fast_exp2(__uint_as_float(sv[e + u]) * sl2 - lse2) : 0.f;
+                        dsv[u] = p * (__uint_as_float(pv[e + u]) - dl);
+                    }
+                    dk[16 * (c & 1) + e / 2] = pack_bf16x2(dsv[0], dsv[1]);
+                }
+                if (c & 1) tmem_st32(tmem + lane_base + kTmS + 32 * (c >> 1), dk);
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(ds_full);
+        }
+        ok = named_bar_and(1, 128, ok);
+        if (ok && n_tiles > 0) {
+            ok = named_bar_and(1, 128, wwait(dq_done, (n_tiles - 1) & 1));
+            tc_fence_after();
+        }
+        if (ok) {
+            const float isd = 1.0f / sqrtf(static_cast<float>(D));
+            float* dst = a.dq + (((size_t)b * nq + tok) * g.H + h) * D;
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t v[32];
+                if (n_tiles > 0) {
+                    tmem_ld32(tmem + lane_base + kTmQ + 32 * c, v);
+                    tmem_ld_wait();
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) v[e] = 0u;
+                }
+                if (row_valid) {
+#pragma unroll
+                    for (int e = 0; e < 32; e += 4)
+                        *reinterpret_cast<float4*>(dst + 32 * c + e) =
+                            make_float4(__uint_as_float(v[e]) * isd, __uint_as_float(v[e + 1]) * isd,
+                                        __uint_as_float(v[e + 2]) * isd, __uint_as_float(v[e + 3]) * isd);
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 5) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+template <class K, class A>
+cudaError_t launch_k(K kernel, const A& args, dim3 grid, size_t smem, cudaStream_t st) {
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    kernel<<<grid, kThreads, smem, st>>>(args);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t attn_bwd_smem_bytes(const Geo& g, int q_frames, int ucap) {
+    const int n_qt = (q_frames * g.nbf + 1) / 2;
+    const size_t a = dkdv_plan(g.D, g.S, n_qt).total + 1024;
+    const size_t b = dq_plan(g.D, g.S, ucap).total + 1024;
+    size_t m = a > b ? a : b;
+    return m < 120 * 1024 ? 120 * 1024 : m;
+}
+
+cudaError_t launch_attn_bwd(const BwdArgs& a, cudaStream_t st) {
+    const Geo& g = a.g;
+    const int nq = a.q_frames * g.tf;
+    const long long nrows = (long long)g.B * nq * g.H;
+    delta_kernel<<<(unsigned)((nrows + 15) / 16), 256, 0, st>>>(a.out, a.dout, a.delta, nq, g.H, g.D, nrows);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+
+    const int qb_total = a.q_frames * g.nbf;
+    DkdvKernelArgs kd;
+    kd.a = a;
+    kd.n_pt_max = (g.S * 8 + 15) / 16;
+    kd.n_qt = (qb_total + 1) / 2;
+    const int n_lt = (a.local_frames * g.nbf + 1) / 2;
+    const size_t smem_kd = attn_bwd_smem_bytes(g, a.q_frames, a.ucap);
+    dim3 grid_kd(kd.n_pt_max + n_lt, g.H, g.B);
+    e = g.D == 128 ? launch_k(dkdv_kernel<128>, kd, grid_kd, smem_kd, st)
+                   : launch_k(dkdv_kernel<64>, kd, grid_kd, smem_kd, st);
+    if (e != cudaSuccess) return e;
+
+    DqKernelArgs kq;
+    kq.a = a;
+    kq.ucap = a.ucap;
+    dim3 grid_q((qb_total + 1) / 2, g.H, g.B);
+    return g.D == 128 ? launch_k(dq_kernel<128>, kq, grid_q, smem_kd, st)
+                      : launch_k(dq_kernel<64>, kq, grid_q, smem_kd, st);
+}
 
 }  // namespace pbsa

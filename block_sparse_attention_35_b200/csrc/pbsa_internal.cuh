@@ -43,6 +43,7 @@ struct BwdArgs {
     Geo g;
     int q_frames, local_frames, ring_head;
     int idx_stride;
+    int ucap;            // capacity of the per-tile union of selections
     const int32_t* pers_len;
     const int32_t* idx;
     const int32_t* cnt;
@@ -72,6 +73,7 @@ cudaError_t launch_attn_fwd(const FwdArgs& a, bool with_mass, cudaStream_t st);
 size_t attn_fwd_smem_bytes(const Geo& g, int ucap);
 
 cudaError_t launch_attn_bwd(const BwdArgs& a, cudaStream_t st);
+size_t attn_bwd_smem_bytes(const Geo& g, int q_frames, int ucap);
 
 cudaError_t launch_cache_update(const Geo& g, const __nv_bfloat16* k_local,
                                 const __nv_bfloat16* v_local, int local_frames, int ring_head,
