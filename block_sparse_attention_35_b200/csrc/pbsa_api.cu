@@ -433,3 +433,41 @@ int pbsa_wait_selftest(int32_t* status, long long timeout_ns, void* stream) {
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------------------------
+// Helpers for entry points defined in other translation units.
+namespace pbsa {
+
+int api_fail(int code, const char* msg) { return fail(code, "%s", msg); }
+
+int api_cuda_fail(cudaError_t e, const char* what) { return cuda_fail(e, what); }
+
+// Checks the arguments of a block selection call exactly as pbsa_select_blocks does and
+// returns the geometry, k, and the bytes of pooled-mean scratch the call needs (query
+// means first, key means at key_offset).
+int api_prepare_select(const pbsa_config* cfg, const void* q, int q_frames, const void* k_local,
+                       int local_frames, int ring_head, const int32_t* idx, int idx_stride,
+                       const int32_t* cnt, const float* scores, Geo* geo, int* k,
+                       size_t* scratch_bytes, size_t* key_offset) {
+    int rc = validate(cfg);
+    if (rc != PBSA_OK) return rc;
+    const Geo g = make_geo(cfg);
+    if ((rc = check_window(cfg, g, q_frames, local_frames, ring_head)) != PBSA_OK) return rc;
+    REQUIRE_PTR(q);
+    REQUIRE_PTR(k_local);
+    REQUIRE_PTR(idx);
+    REQUIRE_PTR(cnt);
+    OPTIONAL_PTR(scores);
+    const int kk = topk_count(cfg, local_frames);
+    if (idx_stride < kk) return fail(PBSA_ERR_ARG, "idx_stride %d < k %d", idx_stride, kk);
+    const int nl = local_frames * g.nbf;
+    if (score_topk_smem_bytes(g, nl) > 227 * 1024)
+        return fail(PBSA_ERR_UNSUPPORTED, "%d local blocks do not fit the scoring kernel", nl);
+    *geo = g;
+    *k = kk;
+    *scratch_bytes = select_ws(g, q_frames);
+    *key_offset = align256(sizeof(float) * (size_t)g.B * g.H * q_frames * g.nbf * g.D);
+    return PBSA_OK;
+}
+
+}  // namespace pbsa

@@ -85,3 +85,13 @@ cudaError_t launch_cache_update(const Geo& g, const __nv_bfloat16* k_local,
 cudaError_t launch_wait_selftest(int32_t* status, long long timeout_ns, cudaStream_t st);
 
 }  // namespace pbsa
+
+namespace pbsa {
+// Shared argument handling for entry points outside pbsa_api.cu.
+int api_fail(int code, const char* msg);
+int api_cuda_fail(cudaError_t e, const char* what);
+int api_prepare_select(const pbsa_config* cfg, const void* q, int q_frames, const void* k_local,
+                       int local_frames, int ring_head, const int32_t* idx, int idx_stride,
+                       const int32_t* cnt, const float* scores, Geo* geo, int* k,
+                       size_t* scratch_bytes, size_t* key_offset);
+}  // namespace pbsa

@@ -213,3 +213,16 @@ def pbsa_cache_update(cfg, k_local, v_local, local_frames, ring_head, mass_local
 
 def pbsa_wait_selftest(status, timeout_ns: int, stream=None):
     _check(_lib.pbsa_wait_selftest(_ptr(status), int(timeout_ns), _stream(stream)))
+
+
+def pbsa_select_blocks_noalloc(cfg, q, q_frames, k_local, local_frames, ring_head, idx,
+                               idx_stride, cnt, scores, stream=None):
+    """Block selection without a workspace, for callers that cannot allocate device
+    memory (the library keeps the scratch in a static device buffer; see include/pbsa.h)."""
+    f = _lib.pbsa_select_blocks_noalloc
+    if f.argtypes is None:
+        P, I = ctypes.c_void_p, ctypes.c_int
+        f.restype = I
+        f.argtypes = [ctypes.POINTER(pbsa_config), P, I, P, I, I, P, I, P, P, P]
+    _check(f(_cfg(cfg), _ptr(q), q_frames, _ptr(k_local), local_frames, ring_head, _ptr(idx),
+             idx_stride, _ptr(cnt), _ptr(scores), _stream(stream)))

@@ -141,6 +141,34 @@ PBSA_API int pbsa_select_blocks(const pbsa_config* cfg, const void* q, int q_fra
                        void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Block selection that allocates nothing and needs no workspace.  The paper has no
+ * counterpart; this is a convenience of this library.
+ *
+ * Some callers cannot allocate device memory where they select blocks: a plugin inside
+ * an inference engine whose memory plan is fixed before it runs, or a decode loop that
+ * must not call cudaMalloc because it blocks the host and synchronises the device.  This
+ * call computes exactly what pbsa_select_blocks computes (same kernels, same results) but
+ * keeps the pooled-mean scratch in a library-owned static device buffer of
+ * PBSA_SELECT_STATIC_SCRATCH_BYTES, held by every GPU that loads the library until exit.
+ *
+ *  - Limit: the scratch a call needs is pbsa_workspace_size(cfg, PBSA_OP_SELECT,
+ *    q_frames); above PBSA_SELECT_STATIC_SCRATCH_BYTES the call returns
+ *    PBSA_ERR_UNSUPPORTED and launches nothing.
+ *  - The first call on a device looks up the buffer's device address (once per device,
+ *    with that device current); make that first call before any stream capture.
+ *  - Every call shares the one buffer.  Calls whose kernels overlap on the GPU (different
+ *    streams, or different host threads on the same device) race on it; order them on
+ *    one stream or with events.  The buffer keeps the last call's contents; nothing in
+ *    it needs clearing between calls.
+ *  - Arguments, layouts and errors are those of pbsa_select_blocks without workspace.
+ */
+#define PBSA_SELECT_STATIC_SCRATCH_BYTES (8u << 20)
+PBSA_API int pbsa_select_blocks_noalloc(const pbsa_config* cfg, const void* q, int q_frames,
+                                        const void* k_local, int local_frames, int ring_head,
+                                        int32_t* idx, int idx_stride, int32_t* cnt,
+                                        float* scores, void* stream);
+
+/*
  * PBSA forward.  (pith.science abstract; project page call attn(query, key_persistent,
  * value_persistent, key_local, value_local).)
  *
