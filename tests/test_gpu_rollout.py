@@ -1,0 +1,101 @@
+"""Rollout with memory updates (decode geometry, 20 chunks of 3 frames, fresh K/V each
+chunk, empty persistent cache at the start): every step runs selection, the forward with
+block mass, the window slide and the persistent merge on the GPU through the C ABI
+(SparseForcingAttention wrapper), and the oracle replays that step from the GPU's state at
+the start of the step.  Index lists, outputs, masses, merge decisions and cache contents
+are compared step by step.  One head keeps the oracle's time low; heads are independent."""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+from block_sparse_attention_35_b200.attention import SparseForcingAttention
+from block_sparse_attention_35_b200.synth import WORKLOADS, rollout_chunk
+from oracle import pbsa_oracle as orc
+from tests.harness import (LSE_ABS, MASS_ABS, MASS_REL, assert_close_bf16, check_topk, f64,
+                           ring_to_window)
+
+pytestmark = pytest.mark.gpu
+
+
+def _logical_mass(ml_phys, ring_head, local_frames, W, nbf):
+    out = np.zeros(ml_phys.shape[:2] + (local_frames * nbf,))
+    for lid in range(local_frames * nbf):
+        out[:, :, lid] = ml_phys[:, :, ((ring_head + lid // nbf) % W) * nbf + lid % nbf]
+    return out
+
+
+def test_rollout_twenty_chunks(cuda_dev):
+    wl = dataclasses.replace(WORKLOADS["rollout"], H=1)
+    a = SparseForcingAttention(wl.B, wl.H, wl.D, wl.frame_h, wl.frame_w, wl.total_cache_size,
+                               wl.local_cache_size, wl.persistent_cache_size,
+                               max_seq_len=wl.max_seq_len,
+                               local_block_sparse_topk_ratio=wl.topk_ratio,
+                               chunk_frames=wl.q_frames, device=cuda_dev)
+    W, tf, nbf, S = a.W, a.tf, a.nbf, a.S
+    exact_frac = []
+    admitted_total = 0
+    for step in range(wl.chunks):
+        q, k, v = rollout_chunk(wl, step)
+        a.append(k.to(cuda_dev), v.to(cuda_dev))
+        qd = q.to(cuda_dev)
+        torch.cuda.synchronize()
+        lf, rh, g0 = a.local_frames, a.ring_head, a.first_frame_global
+        kwin = ring_to_window(a.k_local.cpu(), rh, lf, W, tf)
+        vwin = ring_to_window(a.v_local.cpu(), rh, lf, W, tf)
+        kp, vp = a.k_pers.cpu(), a.v_pers.cpu()
+        plen, pscore0 = a.pers_len.cpu().numpy(), a.pers_score.cpu().double().numpy()
+        ml0 = a.mass_local.cpu().double().numpy()
+
+        a(qd, accumulate_mass=True)
+        torch.cuda.synchronize()
+        assert int(a.status.item()) == 0
+        idx = a.idx.cpu().numpy()
+        # ---- selection
+        idx_o, sc_o = orc.select_blocks(f64(q), f64(kwin), wl.frame_h, wl.frame_w, wl.topk_ratio)
+        kk = idx_o.shape[-1]
+        exact_frac.append(check_topk(idx[..., :kk], a.cnt.cpu().numpy(), sc_o, kk))
+        # ---- forward + mass on the GPU's selection
+        O, lse, mp, ml = orc.attn_fwd(f64(q), f64(kp), f64(vp), plen, f64(kwin), f64(vwin),
+                                      idx[..., :kk], wl.frame_h, wl.frame_w)
+        assert_close_bf16(f64(a.out), O, f"step {step} out")
+        assert np.abs(a.lse.cpu().numpy() - lse).max() <= LSE_ABS
+        ps1 = a.pers_score.cpu().double().numpy()
+        ml1 = a.mass_local.cpu().double().numpy()
+        assert np.allclose(ps1, pscore0 + mp, rtol=MASS_REL, atol=MASS_ABS)
+        assert np.allclose(_logical_mass(ml1, rh, lf, W, nbf),
+                           _logical_mass(ml0, rh, lf, W, nbf) + ml, rtol=MASS_REL, atol=MASS_ABS)
+        # ---- slide + merge
+        n_ev = max(0, lf + wl.q_frames - W)
+        src0 = a.pers_src.cpu().numpy()
+        if n_ev:
+            ml_log = _logical_mass(ml1, rh, lf, W, nbf)
+            # decisions on the GPU's own masses must match exactly
+            r = orc.cache_update(f64(kp), f64(vp), plen, a.pers_score.cpu().double().numpy(),
+                                 src0, f64(kwin), f64(vwin), ml_log, n_ev, g0,
+                                 wl.frame_h, wl.frame_w)
+            # and on the oracle's masses wherever the keep/drop margin exceeds 1e-3
+            cand = [ps1[0, 0, s] for s in range(S) if plen[0, 0, s] > 0] + list(ml_log[0, 0, :n_ev * nbf])
+            srt = sorted(cand, reverse=True)
+            margin = (srt[S - 1] - srt[S]) if len(srt) > S else np.inf
+            a.slide(n_ev)
+            torch.cuda.synchronize()
+            nup = int(a.n_upd[0, 0].item())
+            ups = [tuple(x) for x in a.upd[0, 0, :nup].cpu().numpy()]
+            assert ups == r["updates"][0][0], f"step {step}"
+            assert np.array_equal(a.pers_len.cpu().numpy(), r["pers_len"])
+            assert np.array_equal(a.pers_src.cpu().numpy(), r["pers_src"])
+            assert np.array_equal(f64(a.k_pers), r["k_pers"])
+            assert np.array_equal(f64(a.v_pers), r["v_pers"])
+            if margin > 1e-3:
+                r2 = orc.cache_update(f64(kp), f64(vp), plen, pscore0 + mp, src0, f64(kwin),
+                                      f64(vwin), _logical_mass(ml0, rh, lf, W, nbf) + ml, n_ev,
+                                      g0, wl.frame_h, wl.frame_w)
+                assert r2["updates"][0][0] == ups, f"step {step}: decision differs at margin {margin}"
+            admitted_total += nup
+    # the persistent cache filled up and then kept changing
+    assert int((a.pers_len > 0).sum().item()) == S
+    assert admitted_total > S
+    print(f"rollout: exact top-k fraction per step {np.round(exact_frac, 3).tolist()}, "
+          f"admissions {admitted_total}")
