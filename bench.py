@@ -225,9 +225,11 @@ def make_sets(n, dev, with_bwd):
                                    local_block_sparse_topk_ratio=WL.topk_ratio,
                                    chunk_frames=WL.q_frames, device=dev)
         if shared is None:
-            shared = (a.ws_select, a.ws_fwd, a.ws_bwd)
+            if with_bwd:   # gradient outputs, allocated once, outside any timed region
+                a.backward_buffers()
+            shared = (a.ws_select, a.ws_fwd, a.ws_bwd, a._grads)
         else:
-            a.ws_select, a.ws_fwd, a.ws_bwd = shared
+            a.ws_select, a.ws_fwd, a.ws_bwd, a._grads = shared
         inp = decode_inputs(WL, seed=WL.seed + 100 + s)
         a.k_local.copy_(inp["k_local"])
         a.v_local.copy_(inp["v_local"])

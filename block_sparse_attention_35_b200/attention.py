@@ -126,9 +126,9 @@ class SparseForcingAttention:
         self.select(q)
         return self.attend(q, accumulate_mass)
 
-    def backward(self, q: torch.Tensor, dout: torch.Tensor):
-        """Gradients of sum(out * dout) for the last forward (same caches, same selection).
-        Returns (dq, dk_pers, dv_pers, dk_local, dv_local), fp32, owned by this object."""
+    def backward_buffers(self):
+        """The fp32 gradient outputs (dq, dk_pers, dv_pers, dk_local, dv_local), allocated
+        on first use."""
         if self._grads is None:
             f32 = dict(dtype=torch.float32, device=self.device)
             self._grads = (torch.zeros(self.out.shape, **f32),
@@ -136,7 +136,12 @@ class SparseForcingAttention:
                            torch.zeros(self.v_pers.shape, **f32),
                            torch.zeros(self.k_local.shape, **f32),
                            torch.zeros(self.v_local.shape, **f32))
-        dq, dkp, dvp, dkl, dvl = self._grads
+        return self._grads
+
+    def backward(self, q: torch.Tensor, dout: torch.Tensor):
+        """Gradients of sum(out * dout) for the last forward (same caches, same selection).
+        Returns (dq, dk_pers, dv_pers, dk_local, dv_local), fp32, owned by this object."""
+        dq, dkp, dvp, dkl, dvl = self.backward_buffers()
         P.pbsa_attn_bwd(self.cfg, q, self.chunk_frames, self.k_pers, self.v_pers, self.pers_len,
                         self.k_local, self.v_local, self.local_frames, self.ring_head, self.idx,
                         self.kmax, self.cnt, self.out, self.lse, dout, dq, dkp, dvp, dkl, dvl,

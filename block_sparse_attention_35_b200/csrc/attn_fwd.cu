@@ -7,26 +7,26 @@
 // probability summed over the chunk's query rows (the score that ranks blocks when the
 // window slides).
 //
-// One CTA = one 128-row query tile = two 8x8 query blocks of one (batch, head), each
-// loaded as a 64-row 5-D TMA box [1 frame, 8 rows, 8 cols, 1 head, 64 channels]; rows of
-// ragged edge blocks fall outside the tensor and are zero-filled on load and clipped on
-// store.  Key tiles are 128 keys:
-//   * persistent phase: the occupied slots' valid rows, compacted into a stream of 8-row
-//     groups (slot lengths are multiples of 8), 16 groups per tile, each group one 2-D TMA
-//     box; only the last tile is partial;
-//   * local phase: the union of the two query blocks' selections, two 8x8 key blocks per
-//     tile, each a 5-D TMA box from the ring; columns of a block the row's query block did
-//     not select, or outside the frame, are masked.
-// Warp roles (192 threads): warps 0-3 softmax (one query row per thread), warp 4 TMA
-// producer, warp 5 MMA issuer.  TMEM: S double buffer (2 x 128 columns) and the O
-// accumulator (D columns).  S = Q K^T is an SS MMA (both operands K-major, 128-byte
-// swizzle); P is converted to bf16 in registers and written back over S in TMEM, and
-// O += P V is a TS MMA (A from TMEM, V MN-major in shared memory).  O is rescaled only
-// when a row maximum grows by more than 2^8 (exponentials stay <= 256).
-// Mass: while streaming, each row emits for every slot/block it saw the log2 of its
-// partial probability sum (relative to the running maximum) into per-CTA scratch; after
-// the final log-sum-exp is known the CTA turns them into probabilities, sums over rows
-// and adds one value per slot/block to the global mass arrays.
+// One CTA = four 8x8 query blocks of one (batch, head), split into two 128-row query tiles
+// ("sides" A and B, two blocks each, every block a 64-row 5-D TMA box; ragged edge blocks
+// are zero-filled on load and clipped on store).  Key tiles are 128 keys:
+//   * persistent tiles (shared by both sides): the occupied slots' valid rows compacted
+//     into a stream of 8-row groups (slot lengths are multiples of 8), 16 groups per tile;
+//   * local tiles (one side each): the union of that side's two selections, two 8x8 key
+//     blocks per tile; columns the row's query block did not select, or outside the frame,
+//     are masked.  A-tiles and B-tiles alternate in the stream.
+// TMEM (512 columns): S_A | S_B | O_A | O_B.  P (bf16) is written over the first 64 columns
+// of its S and read by a TS MMA; the tensor pipe executes one thread's MMAs in issue order,
+// so S = Q K^T of a side's next tile may be issued right after the O += P V that reads
+// its P.  Issue order per persistent tile: QK_A(t), PV_B(t-1), QK_B(t), PV_A(t), so each
+// side's softmax of tile t runs while the other side's MMAs occupy the tensor pipe.
+// Warp roles (384 threads): warps 0-3 softmax of side A, 4-7 side B (one query row per
+// thread), warp 8 K (and Q) producer, warp 9 V producer, warp 10 MMA issuer, warp 11 idle.  K and V
+// stages have separate full/empty barriers.  O is rescaled only when a row maximum grows by
+// more than 2^8.  Mass: each row emits, per slot/block it saw, log2 of its partial
+// probability sum (relative to its running maximum) into workspace; once the final
+// log-sum-exp is known the side converts them, sums over its rows and adds one value per
+// slot/block to the global mass arrays.
 #include <cuda_bf16.h>
 #include <math_constants.h>
 
@@ -37,10 +37,17 @@ namespace pbsa {
 
 namespace {
 
-constexpr int kNst = 2;               // K/V pipeline stages
-constexpr uint32_t kHalf = 128 * 128; // bytes of 128 rows x 64 bf16 channels
-constexpr uint32_t kTmS0 = 0, kTmS1 = 128, kTmO = 256, kTmCols = 512;
-constexpr int kThreads = 192;
+constexpr int kNst = 2;                // K and V pipeline stages
+constexpr uint32_t kHalf = 128 * 128;  // bytes of 128 rows x 64 bf16 channels
+constexpr uint32_t kTmCols = 512;
+constexpr int kThreads = 384;
+// Register split: the kernel launches at kLaunchRegs per thread (384 x 168 = 64512); the
+// producer/MMA warpgroup drops to kRegsIo and both softmax warpgroups rise to kRegsSoftmax,
+// 2 x 128 x 200 + 128 x 104 = 64512, exactly the launch pool.  The host refuses to launch if
+// ptxas did not give the kernel kLaunchRegs, so the increase can always be satisfied.
+constexpr int kLaunchRegs = 168, kRegsIo = 104, kRegsSoftmax = 200;
+static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsIo <= kThreads * kLaunchRegs, "register split");
+constexpr float kLog2e = 1.4426950408889634f;
 
 struct SmemPlan {
     uint32_t q, k, v, grp_row, grp_seg, seg_slot, uni_blk, uni_bits, seg_mass, bars, misc,
@@ -50,30 +57,31 @@ struct SmemPlan {
 __host__ __device__ inline SmemPlan fwd_plan(int D, int S, int ucap) {
     SmemPlan p;
     const uint32_t nh = D / 64;
-    p.q = 0;
-    p.k = p.q + nh * kHalf;
+    p.q = 0;                                 // 2 sides
+    p.k = p.q + 2 * nh * kHalf;
     p.v = p.k + kNst * nh * kHalf;
     p.grp_row = p.v + kNst * nh * kHalf;
     p.grp_seg = p.grp_row + 4u * 8u * S;
     p.seg_slot = p.grp_seg + 4u * 8u * S;
-    p.uni_blk = p.seg_slot + 4u * S;
-    p.uni_bits = p.uni_blk + 4u * ucap;
-    p.seg_mass = p.uni_bits + 4u * ucap;
-    p.bars = (p.seg_mass + 4u * (S + ucap) + 7u) & ~7u;
-    p.misc = p.bars + 8u * 16u;
-    p.total = p.misc + 4u * 8u;
+    p.uni_blk = p.seg_slot + 4u * S;         // [2][ucap]
+    p.uni_bits = p.uni_blk + 8u * ucap;      // [2][ucap]
+    p.seg_mass = p.uni_bits + 8u * ucap;     // [2][S + ucap]
+    p.bars = (p.seg_mass + 8u * (S + ucap) + 7u) & ~7u;
+    p.misc = p.bars + 8u * 24u;
+    p.total = p.misc + 4u * 16u;
     return p;
 }
 
 // barrier slots
-enum { B_Q = 0, B_KF = 1, B_VF = 3, B_KE = 5, B_SF = 7, B_PF = 9, B_PV = 11, B_DRAIN = 13 };
+enum {
+    B_Q = 0, B_KF = 1, B_KE = 3, B_VF = 5, B_VE = 7, B_SF = 9, B_PF = 11, B_PV = 13, B_DRAIN = 15
+};
 // misc slots
-enum { M_TMEM = 0, M_ABORT = 1, M_G = 2, M_OCC = 3, M_U = 4 };
+enum { M_TMEM = 0, M_ABORT = 1, M_G = 2, M_OCC = 3, M_UA = 4, M_UB = 5 };
 
 struct FwdKernelArgs {
     FwdArgs a;
-    int ucap;
-    int n_ctiles;  // query tiles per (b, h)
+    int n_groups;  // CTAs per (b, h): ceil(QB / 4)
 };
 
 __device__ __forceinline__ float warp_sum(float v) {
@@ -82,17 +90,62 @@ __device__ __forceinline__ float warp_sum(float v) {
     return v;
 }
 
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// (a.x * s - m, a.y * s - m) on the packed fp32x2 pipe
+__device__ __forceinline__ float2 ffma2(float2 a, float s, float m) {
+    uint64_t r;
+    const uint64_t av = (static_cast<uint64_t>(__float_as_uint(a.y)) << 32) | __float_as_uint(a.x);
+    const uint64_t sv = (static_cast<uint64_t>(__float_as_uint(s)) << 32) | __float_as_uint(s);
+    const uint64_t mv = (static_cast<uint64_t>(__float_as_uint(-m)) << 32) | __float_as_uint(-m);
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(av), "l"(sv), "l"(mv));
+    return make_float2(__uint_as_float(static_cast<uint32_t>(r)), __uint_as_float(static_cast<uint32_t>(r >> 32)));
+}
+
+// 64-bit validity mask of one 8x8 key block: rows < hv, columns < wv, all zero if !sel.
+__device__ __forceinline__ uint64_t block_mask(bool sel, int hv, int wv) {
+    if (!sel) return 0ull;
+    const uint64_t rows = hv >= 8 ? ~0ull : ((1ull << (8 * hv)) - 1ull);
+    const uint64_t cols = 0x0101010101010101ull * static_cast<uint64_t>((1u << wv) - 1u);
+    return rows & cols;
+}
+
+__device__ __forceinline__ uint64_t prefix_mask(int n) {  // bits [0, n), n in [0, 64]
+    return n >= 64 ? ~0ull : ((1ull << n) - 1ull);
+}
+
+// Consumers of stream tile t: bit 0 = side A, bit 1 = side B; *lj = local tile index.
+// Persistent tiles come first (both sides), then the sides' local tiles alternate A, B.
+__device__ __forceinline__ int tile_cons(int t, int n_pt, int nla, int nlb, bool has_b, int* lj) {
+    if (t < n_pt) {
+        *lj = -1;
+        return has_b ? 3 : 1;
+    }
+    const int j = t - n_pt, m = min(nla, nlb);
+    if (j < 2 * m) {
+        *lj = j >> 1;
+        return (j & 1) ? 2 : 1;
+    }
+    *lj = m + (j - 2 * m);
+    return nla > nlb ? 1 : 2;
+}
+
 template <int D, bool MASS>
 __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_constant__ FwdKernelArgs ka) {
     constexpr int NH = D / 64;
     constexpr uint32_t KV_BYTES = NH * kHalf;
+    constexpr uint32_t Q_SIDE = NH * kHalf;
     const FwdArgs& a = ka.a;
     const Geo& g = a.g;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
     const int S = g.S;
-    const int ucap = ka.ucap;
+    const int ucap = a.ucap;
     const SmemPlan P = fwd_plan(D, S, ucap);
     uint8_t* sQ = sm + P.q;
     uint8_t* sK = sm + P.k;
@@ -107,32 +160,37 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     int* misc = reinterpret_cast<int*>(sm + P.misc);
     volatile int* abort_flag = misc + M_ABORT;
 
-    const int tile = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int grp = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int bh = b * g.H + h;
     const int qb_total = a.q_frames * g.nbf;
-    const int qb0 = 2 * tile;
-    const int qb1 = (2 * tile + 1 < qb_total) ? 2 * tile + 1 : -1;
     const int nl = a.local_frames * g.nbf;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // query blocks of the two sides (-1 = none)
+    auto qblock = [&](int X, int i) -> int {
+        const int qb = 4 * grp + 2 * X + i;
+        return qb < qb_total ? qb : -1;
+    };
+    const bool has_b = qblock(1, 0) >= 0;
 
     // ------------------------------------------------------------------ set-up
     if (threadIdx.x == 0) {
         mbar_init(&bars[B_Q], 1);
         for (int s = 0; s < kNst; ++s) {
             mbar_init(&bars[B_KF + s], 1);
-            mbar_init(&bars[B_VF + s], 1);
             mbar_init(&bars[B_KE + s], 1);
+            mbar_init(&bars[B_VF + s], 1);
+            mbar_init(&bars[B_VE + s], 1);
         }
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(&bars[B_SF + s], 1);
-            mbar_init(&bars[B_PF + s], 128);
-            mbar_init(&bars[B_PV + s], 1);
+        for (int x = 0; x < 2; ++x) {
+            mbar_init(&bars[B_SF + x], 1);
+            mbar_init(&bars[B_PF + x], 128);
+            mbar_init(&bars[B_PV + x], 1);
         }
         mbar_init(&bars[B_DRAIN], 1);
         misc[M_ABORT] = 0;
         fence_barrier_init();
     }
-    if (warp == 5) tmem_alloc(reinterpret_cast<uint32_t*>(misc + M_TMEM), kTmCols);
+    if (warp == 10) tmem_alloc(reinterpret_cast<uint32_t*>(misc + M_TMEM), kTmCols);
     if (warp == 0) {
         // compacted stream of the occupied slots' 8-row groups
         int run = 0, occ = 0;
@@ -170,185 +228,208 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
             misc[M_OCC] = occ;
         }
     }
-    if (warp == 1 && lane == 0) {
-        // union of the two query blocks' selections (both lists ascending)
-        const int c0 = min(max(a.cnt[(size_t)bh * qb_total + qb0], 0), a.idx_stride);
-        const int c1 = qb1 >= 0 ? min(max(a.cnt[(size_t)bh * qb_total + qb1], 0), a.idx_stride) : 0;
-        const int32_t* i0 = a.idx + ((size_t)bh * qb_total + qb0) * a.idx_stride;
-        const int32_t* i1 = a.idx + ((size_t)bh * qb_total + (qb1 >= 0 ? qb1 : qb0)) * a.idx_stride;
-        int p = 0, q = 0, u = 0;
-        while (p < c0 || q < c1) {
-            if (u == ucap) {
-                set_status(a.status, PBSA_ERR_DEVICE_CHECK);
-                break;
+    if ((warp == 1 || warp == 2) && lane == 0) {
+        // union of one side's two selections (both lists ascending)
+        const int X = warp - 1;
+        const int q0 = qblock(X, 0), q1 = qblock(X, 1);
+        int u = 0;
+        if (q0 >= 0) {
+            const int c0 = min(max(a.cnt[(size_t)bh * qb_total + q0], 0), a.idx_stride);
+            const int c1 = q1 >= 0 ? min(max(a.cnt[(size_t)bh * qb_total + q1], 0), a.idx_stride) : 0;
+            const int32_t* i0 = a.idx + ((size_t)bh * qb_total + q0) * a.idx_stride;
+            const int32_t* i1 = a.idx + ((size_t)bh * qb_total + (q1 >= 0 ? q1 : q0)) * a.idx_stride;
+            int p = 0, q = 0;
+            while (p < c0 || q < c1) {
+                if (u == ucap) {
+                    set_status(a.status, PBSA_ERR_DEVICE_CHECK);
+                    break;
+                }
+                const int v0 = p < c0 ? i0[p] : 0x7fffffff;
+                const int v1 = q < c1 ? i1[q] : 0x7fffffff;
+                int blk, bits;
+                if (v0 == v1) {
+                    blk = v0; bits = 3; ++p; ++q;
+                } else if (v0 < v1) {
+                    blk = v0; bits = 1; ++p;
+                } else {
+                    blk = v1; bits = 2; ++q;
+                }
+                if (blk < 0 || blk >= nl) {
+                    set_status(a.status, PBSA_ERR_DEVICE_CHECK);
+                    continue;
+                }
+                uni_blk[X * ucap + u] = blk;
+                uni_bits[X * ucap + u] = bits;
+                ++u;
             }
-            const int v0 = p < c0 ? i0[p] : 0x7fffffff;
-            const int v1 = q < c1 ? i1[q] : 0x7fffffff;
-            int blk, bits;
-            if (v0 == v1) {
-                blk = v0; bits = 3; ++p; ++q;
-            } else if (v0 < v1) {
-                blk = v0; bits = 1; ++p;
-            } else {
-                blk = v1; bits = 2; ++q;
-            }
-            if (blk < 0 || blk >= nl) {
-                set_status(a.status, PBSA_ERR_DEVICE_CHECK);
-                continue;
-            }
-            uni_blk[u] = blk;
-            uni_bits[u] = bits;
-            ++u;
         }
-        misc[M_U] = u;
+        misc[M_UA + X] = u;
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
 
     const uint32_t tmem = static_cast<uint32_t>(misc[M_TMEM]);
-    const int G = misc[M_G], n_occ = misc[M_OCC], U = misc[M_U];
+    const int G = misc[M_G], n_occ = misc[M_OCC];
+    const int UA = misc[M_UA], UB = misc[M_UB];
     const int n_pt = (G + 15) / 16;
-    const int n_tiles = n_pt + (U + 1) / 2;
+    const int nla = (UA + 1) / 2, nlb = has_b ? (UB + 1) / 2 : 0;
+    const int n_stream = n_pt + nla + nlb;
+    const int n_side0 = n_pt + nla, n_side1 = has_b ? n_pt + nlb : 0;
 
-    if (warp == 4) {
-        // ------------------------------------------------------------ TMA producer
+    if (warp >= 8) {
+      asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsIo));
+      if (warp == 8 || warp == 9) {
+        // ------------------------------------------------- TMA producers (K+Q, V)
         if (lane == 0) {
-            tma_prefetch_desc(&a.tm_q);
-            tma_prefetch_desc(&a.tm_kp);
-            tma_prefetch_desc(&a.tm_vp);
-            tma_prefetch_desc(&a.tm_kl);
-            tma_prefetch_desc(&a.tm_vl);
-            mbar_arrive_expect_tx(&bars[B_Q], 2 * NH * (kHalf / 2));
-            for (int hb = 0; hb < 2; ++hb) {
-                const int qb = (hb == 1 && qb1 >= 0) ? qb1 : qb0;
-                const int f = qb / g.nbf, i = qb % g.nbf;
-                const int by = i / g.nbx, bx = i % g.nbx;
-                for (int hh = 0; hh < NH; ++hh)
-                    tma_load_5d(sQ + hh * kHalf + hb * (kHalf / 2), &a.tm_q, &bars[B_Q], hh * 64, h,
-                                8 * bx, 8 * by, b * a.q_frames + f);
+            const bool isK = warp == 8;
+            const CUtensorMap* mp = isK ? &a.tm_kp : &a.tm_vp;
+            const CUtensorMap* ml = isK ? &a.tm_kl : &a.tm_vl;
+            uint8_t* base = isK ? sK : sV;
+            uint64_t* full = &bars[isK ? B_KF : B_VF];
+            uint64_t* empty = &bars[isK ? B_KE : B_VE];
+            tma_prefetch_desc(mp);
+            tma_prefetch_desc(ml);
+            if (isK) {
+                tma_prefetch_desc(&a.tm_q);
+                mbar_arrive_expect_tx(&bars[B_Q], 2 * 2 * NH * (kHalf / 2));
+                for (int X = 0; X < 2; ++X)
+                    for (int hb = 0; hb < 2; ++hb) {
+                        int qb = qblock(X, hb);
+                        if (qb < 0) qb = qblock(0, 0);  // filler rows, never stored
+                        const int f = qb / g.nbf, i = qb % g.nbf;
+                        for (int hh = 0; hh < NH; ++hh)
+                            tma_load_5d(sQ + X * Q_SIDE + hh * kHalf + hb * (kHalf / 2), &a.tm_q, &bars[B_Q],
+                                        hh * 64, h, 8 * (i % g.nbx), 8 * (i / g.nbx), b * a.q_frames + f);
+                    }
             }
             int issued = 0;
-            for (int it = 0; it < n_tiles; ++it) {
-                const int st = it % kNst;
-                if (it >= kNst &&
-                    !mbar_wait(&bars[B_KE + st], ((it / kNst) - 1) & 1, abort_flag, a.status))
-                    break;
-                uint8_t* dk = sK + st * KV_BYTES;
-                uint8_t* dv = sV + st * KV_BYTES;
-                mbar_arrive_expect_tx(&bars[B_KF + st], KV_BYTES);
-                if (it < n_pt) {
+            for (int t = 0; t < n_stream; ++t) {
+                const int st = t % kNst;
+                if (t >= kNst && !mbar_wait(&empty[st], ((t / kNst) - 1) & 1, abort_flag, a.status)) break;
+                uint8_t* dst = base + st * KV_BYTES;
+                mbar_arrive_expect_tx(&full[st], KV_BYTES);
+                int lj;
+                const int cons = tile_cons(t, n_pt, nla, nlb, has_b, &lj);
+                if (lj < 0) {
                     for (int c = 0; c < 16; ++c) {
-                        const int row = grp_row[min(it * 16 + c, G - 1)];
+                        const int row = grp_row[min(t * 16 + c, G - 1)];
                         for (int hh = 0; hh < NH; ++hh)
-                            tma_load_2d(dk + hh * kHalf + c * 1024, &a.tm_kp, &bars[B_KF + st],
-                                        hh * 64, row);
-                    }
-                    mbar_arrive_expect_tx(&bars[B_VF + st], KV_BYTES);
-                    for (int c = 0; c < 16; ++c) {
-                        const int row = grp_row[min(it * 16 + c, G - 1)];
-                        for (int hh = 0; hh < NH; ++hh)
-                            tma_load_2d(dv + hh * kHalf + c * 1024, &a.tm_vp, &bars[B_VF + st],
-                                        hh * 64, row);
+                            tma_load_2d(dst + hh * kHalf + c * 1024, mp, &full[st], hh * 64, row);
                     }
                 } else {
-                    const int j = it - n_pt;
-                    int crd[2][3];
+                    const int X = cons == 2 ? 1 : 0;
+                    const int U = X ? UB : UA;
                     for (int hb = 0; hb < 2; ++hb) {
-                        const int L = uni_blk[min(2 * j + hb, U - 1)];
+                        const int L = uni_blk[X * ucap + min(2 * lj + hb, U - 1)];
                         const int pos = L / g.nbf, i = L % g.nbf;
-                        crd[hb][0] = 8 * (i % g.nbx);
-                        crd[hb][1] = 8 * (i / g.nbx);
-                        crd[hb][2] = b * g.W + (a.ring_head + pos) % g.W;
+                        const int cf = b * g.W + (a.ring_head + pos) % g.W;
+                        for (int hh = 0; hh < NH; ++hh)
+                            tma_load_5d(dst + hh * kHalf + hb * (kHalf / 2), ml, &full[st], hh * 64, h,
+                                        8 * (i % g.nbx), 8 * (i / g.nbx), cf);
                     }
-                    for (int hb = 0; hb < 2; ++hb)
-                        for (int hh = 0; hh < NH; ++hh)
-                            tma_load_5d(dk + hh * kHalf + hb * (kHalf / 2), &a.tm_kl,
-                                        &bars[B_KF + st], hh * 64, h, crd[hb][0], crd[hb][1],
-                                        crd[hb][2]);
-                    mbar_arrive_expect_tx(&bars[B_VF + st], KV_BYTES);
-                    for (int hb = 0; hb < 2; ++hb)
-                        for (int hh = 0; hh < NH; ++hh)
-                            tma_load_5d(dv + hh * kHalf + hb * (kHalf / 2), &a.tm_vl,
-                                        &bars[B_VF + st], hh * 64, h, crd[hb][0], crd[hb][1],
-                                        crd[hb][2]);
                 }
                 ++issued;
             }
             if (*abort_flag) {
                 // let the copies already issued land before the CTA leaves
-                mbar_wait_drain(&bars[B_Q], 0, 100000000ull);
-                for (int it = max(0, issued - kNst); it < issued; ++it) {
-                    const int st = it % kNst;
-                    mbar_wait_drain(&bars[B_KF + st], (it / kNst) & 1, 100000000ull);
-                    mbar_wait_drain(&bars[B_VF + st], (it / kNst) & 1, 100000000ull);
-                }
+                if (isK) mbar_wait_drain(&bars[B_Q], 0, 100000000ull);
+                for (int t = max(0, issued - kNst); t < issued; ++t)
+                    mbar_wait_drain(&full[t % kNst], (t / kNst) & 1, 100000000ull);
             }
         }
-    } else if (warp == 5) {
+    } else if (warp == 10) {
         // ------------------------------------------------------------- MMA issuer
         if (lane == 0) {
             constexpr uint32_t idesc_qk = idesc_bf16(128, 128, false, false);
             constexpr uint32_t idesc_pv = idesc_bf16(128, D, false, true);
-            const uint32_t q_base = smem_u32(sQ);
             bool ok = mbar_wait(&bars[B_Q], 0, abort_flag, a.status);
-            auto issue_pv = [&](int j) -> bool {
-                const int sbj = j & 1, stj = j % kNst;
-                if (!mbar_wait(&bars[B_PF + sbj], (j >> 1) & 1, abort_flag, a.status)) return false;
-                if (!mbar_wait(&bars[B_VF + stj], (j / kNst) & 1, abort_flag, a.status)) return false;
+            int pend[2] = {-1, -1};    // stream tile whose PV is still to be issued, per side
+            int nqk[2] = {0, 0};       // QK MMAs issued per side
+            int npv[2] = {0, 0};       // PV MMAs issued per side
+            int vrem[kNst] = {0, 0};   // PVs still to read each V stage
+            const int n_side[2] = {n_side0, n_side1};
+            auto issue_pv = [&](int X) -> bool {
+                const int t = pend[X], st = t % kNst;
+                if (!mbar_wait(&bars[B_PF + X], npv[X] & 1, abort_flag, a.status)) return false;
+                if (!mbar_wait(&bars[B_VF + st], (t / kNst) & 1, abort_flag, a.status)) return false;
                 tc_fence_after();
-                const uint32_t p_tmem = tmem + (sbj ? kTmS1 : kTmS0);
-                const uint32_t v_base = smem_u32(sV + stj * KV_BYTES);
+                const uint32_t p_tmem = tmem + 128 * X;
+                const uint32_t o_tmem = tmem + 256 + 128 * X;
+                const uint32_t v_base = smem_u32(sV + st * KV_BYTES);
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint64_t bdesc = sdesc_sw128(v_base + kk * 2048, kHalf, 1024);
-                    umma_ts(tmem + kTmO, p_tmem + kk * 8, bdesc, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
-                }
-                umma_commit(&bars[B_PV + sbj]);
-                umma_commit(&bars[B_KE + stj]);
+                for (int kk = 0; kk < 8; ++kk)
+                    umma_ts(o_tmem, p_tmem + kk * 8, sdesc_sw128(v_base + kk * 2048, kHalf, 1024), idesc_pv,
+                            (npv[X] > 0 || kk > 0) ? 1u : 0u);
+                umma_commit(&bars[B_PV + X]);
+                ++npv[X];
+                if (--vrem[st] == 0) umma_commit(&bars[B_VE + st]);
+                pend[X] = -1;
                 return true;
             };
-            for (int it = 0; ok && it < n_tiles; ++it) {
-                const int st = it % kNst, sb = it & 1;
-                if (!mbar_wait(&bars[B_KF + st], (it / kNst) & 1, abort_flag, a.status)) { ok = false; break; }
-                if (it >= 2 && !mbar_wait(&bars[B_PV + sb], ((it - 2) >> 1) & 1, abort_flag, a.status)) { ok = false; break; }
-                tc_fence_after();
-                const uint32_t s_tmem = tmem + (sb ? kTmS1 : kTmS0);
+            for (int t = 0; ok && t < n_stream; ++t) {
+                const int st = t % kNst;
+                if (!mbar_wait(&bars[B_KF + st], (t / kNst) & 1, abort_flag, a.status)) { ok = false; break; }
+                int lj;
+                const int cons = tile_cons(t, n_pt, nla, nlb, has_b, &lj);
                 const uint32_t k_base = smem_u32(sK + st * KV_BYTES);
+                for (int X = 0; X < 2; ++X) {
+                    if (cons & (1 << X)) {
+                        if (pend[X] >= 0 && !issue_pv(X)) { ok = false; break; }
+                        tc_fence_after();
+                        const uint32_t q_base = smem_u32(sQ + X * Q_SIDE);
+                        const uint32_t s_tmem = tmem + 128 * X;
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
-                    const uint64_t adesc = sdesc_sw128(q_base + off, 16, 1024);
-                    const uint64_t bdesc = sdesc_sw128(k_base + off, 16, 1024);
-                    umma_ss(s_tmem, adesc, bdesc, idesc_qk, kk > 0 ? 1u : 0u);
+                        for (int kk = 0; kk < D / 16; ++kk) {
+                            const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
+                            umma_ss(s_tmem, sdesc_sw128(q_base + off, 16, 1024), sdesc_sw128(k_base + off, 16, 1024),
+                                    idesc_qk, kk > 0 ? 1u : 0u);
+                        }
+                        umma_commit(&bars[B_SF + X]);
+                        ++nqk[X];
+                        pend[X] = t;
+                    } else if (pend[X] >= 0 && nqk[X] == n_side[X]) {
+                        // this side has no more tiles: finish it now so its V stage frees up
+                        if (!issue_pv(X)) { ok = false; break; }
+                    }
                 }
-                umma_commit(&bars[B_SF + sb]);
-                if (it >= 1 && !issue_pv(it - 1)) { ok = false; break; }
+                if (!ok) break;
+                umma_commit(&bars[B_KE + st]);
+                vrem[st] = __popc(cons);
             }
-            if (ok && n_tiles > 0) ok = issue_pv(n_tiles - 1);
+            for (int X = 0; ok && X < 2; ++X)
+                if (pend[X] >= 0 && !issue_pv(X)) ok = false;
             if (!ok) {
                 // wait for the MMAs already issued before TMEM is released
                 umma_commit(&bars[B_DRAIN]);
                 mbar_wait_drain(&bars[B_DRAIN], 0, 100000000ull);
             }
         }
+      }
     } else {
-        // --------------------------------------------------------- softmax warps
-        const int r = threadIdx.x;  // query row of the tile = TMEM lane
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
+        // ------------------------------------------------------ softmax warpgroups
+        const int X = warp >> 2;          // side
+        const int r = threadIdx.x & 127;  // query row of the side's tile = TMEM lane
+        const int wq = warp & 3;          // lane quarter
+        const int nX = X ? n_side1 : n_side0;
         const int hq = r >> 6, rr = r & 63, dy = rr >> 3, dx = rr & 7;
-        const int qbr = hq ? qb1 : qb0;
-        const int qbv = qbr >= 0 ? qbr : qb0;
+        const int qbr = qblock(X, hq);
+        const int qbv = qbr >= 0 ? qbr : 0;
         const int qf = qbv / g.nbf, qi = qbv % g.nbf;
         const int qy = 8 * (qi / g.nbx) + dy, qx = 8 * (qi % g.nbx) + dx;
         const bool row_valid = qbr >= 0 && qy < g.fh && qx < g.fw;
-        const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-        const float sl2 = 1.4426950408889634f / sqrtf(static_cast<float>(D));
+        const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
+        const uint32_t s_col = 128 * X, o_col = 256 + 128 * X;
+        const float sl2 = kLog2e / sqrtf(static_cast<float>(D));
+        const int U = X ? UB : UA;
+        const int32_t* ublk = uni_blk + X * ucap;
+        const int32_t* ubits = uni_bits + X * ucap;
         const size_t scratch_base =
-            ((size_t)(bh * ka.n_ctiles + tile) * a.n_seg_max) * 128 + r;
+            (((size_t)(bh * ka.n_groups + grp) * 2 + X) * a.n_seg_max) * 128 + r;
         float m = -CUDART_INF_F, l = 0.f, carry = 0.f;
         int cur_seg = -1;
         bool ok = true;
-        // every wait result is made warp-uniform: tcgen05.ld/st are warp-collective
         auto wwait = [&](uint64_t* bar, uint32_t parity) -> bool {
             return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, a.status));
         };
@@ -356,60 +437,73 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
             if (MASS) a.scratch[scratch_base + (size_t)seg * 128] = v > 0.f ? mu + fast_log2(v) : -CUDART_INF_F;
         };
 
-        for (int it = 0; it < n_tiles; ++it) {
-            const int sb = it & 1;
-            if (!wwait(&bars[B_SF + sb], (it >> 1) & 1)) { ok = false; break; }
+        for (int k = 0; k < nX; ++k) {
+            if (!wwait(&bars[B_SF + X], k & 1)) { ok = false; break; }
             tc_fence_after();
-            const uint32_t s_addr = tmem + lane_base + (sb ? kTmS1 : kTmS0);
+            const uint32_t s_addr = tmem + lane_base + s_col;
             float x[128];
             {
-                uint32_t v[32];
+                uint32_t v[4][32];
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    tmem_ld32(s_addr + 32 * c, v);
-                    tmem_ld_wait();
+                for (int c = 0; c < 4; ++c) tmem_ld32(s_addr + 32 * c, v[c]);
+                tmem_ld_wait();
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) x[32 * c + e] = __uint_as_float(v[e]);
+                for (int c = 0; c < 4; ++c)
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) x[32 * c + e] = __uint_as_float(v[c][e]);
+            }
+            const bool persistent = k < n_pt;
+            int lj = 0;
+            bool masked;
+            uint64_t mk0 = ~0ull, mk1 = ~0ull;
+            if (persistent) {
+                const int nvc = min(128, 8 * (G - 16 * k));
+                masked = nvc < 128;
+                if (masked) {
+                    mk0 = prefix_mask(min(nvc, 64));
+                    mk1 = prefix_mask(max(nvc - 64, 0));
+                }
+            } else {
+                lj = k - n_pt;
+                const int u0 = 2 * lj;
+                const bool has1 = u0 + 1 < U;
+                const int L0 = ublk[u0], L1 = has1 ? ublk[u0 + 1] : L0;
+                const bool sel0 = (ubits[u0] >> hq) & 1;
+                const bool sel1 = has1 && ((ubits[u0 + 1] >> hq) & 1);
+                const int i0 = L0 % g.nbf, i1 = L1 % g.nbf;
+                mk0 = block_mask(sel0, min(8, g.fh - 8 * (i0 / g.nbx)), min(8, g.fw - 8 * (i0 % g.nbx)));
+                mk1 = block_mask(sel1, min(8, g.fh - 8 * (i1 / g.nbx)), min(8, g.fw - 8 * (i1 % g.nbx)));
+                masked = true;
+            }
+            if (masked) {
+#pragma unroll
+                for (int c = 0; c < 64; ++c) {
+                    if (!((mk0 >> c) & 1ull)) x[c] = -CUDART_INF_F;
+                    if (!((mk1 >> c) & 1ull)) x[64 + c] = -CUDART_INF_F;
                 }
             }
-            // masks -> x in log2 units, -inf where masked
-            if (it < n_pt) {
-                const int nvc = min(128, 8 * (G - 16 * it));
+            // row maximum of the raw scores (tree of 3-input max)
+            float mx[8];
 #pragma unroll
-                for (int c = 0; c < 128; ++c) x[c] = (c < nvc) ? x[c] * sl2 : -CUDART_INF_F;
-            } else {
-                const int j = it - n_pt;
-                const int u0 = 2 * j;
-                const bool has1 = u0 + 1 < U;
-                const int L0 = uni_blk[u0], L1 = has1 ? uni_blk[u0 + 1] : L0;
-                const bool sel0 = (uni_bits[u0] >> hq) & 1;
-                const bool sel1 = has1 && ((uni_bits[u0 + 1] >> hq) & 1);
-                const int i0 = L0 % g.nbf, i1 = L1 % g.nbf;
-                const int hv0 = sel0 ? min(8, g.fh - 8 * (i0 / g.nbx)) : 0;
-                const int wv0 = min(8, g.fw - 8 * (i0 % g.nbx));
-                const int hv1 = sel1 ? min(8, g.fh - 8 * (i1 / g.nbx)) : 0;
-                const int wv1 = min(8, g.fw - 8 * (i1 % g.nbx));
+            for (int j = 0; j < 8; ++j) mx[j] = x[j];
 #pragma unroll
-                for (int c = 0; c < 64; ++c)
-                    x[c] = ((c >> 3) < hv0 && (c & 7) < wv0) ? x[c] * sl2 : -CUDART_INF_F;
+            for (int c = 8; c + 16 <= 128; c += 16)
 #pragma unroll
-                for (int c = 0; c < 64; ++c)
-                    x[64 + c] = ((c >> 3) < hv1 && (c & 7) < wv1) ? x[64 + c] * sl2 : -CUDART_INF_F;
-            }
-            float mt = x[0];
+                for (int j = 0; j < 8; ++j) mx[j] = max3f(mx[j], x[c + j], x[c + 8 + j]);
+            float mt = max3f(max3f(mx[0], mx[1], mx[2]), max3f(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
 #pragma unroll
-            for (int c = 1; c < 128; ++c) mt = fmaxf(mt, x[c]);
-            const float m_new = fmaxf(m, mt);
+            for (int c = 120; c < 128; ++c) mt = fmaxf(mt, x[c]);
+            const float m_new = fmaxf(m, mt * sl2);
             const bool need = m_new > m + 8.0f;
             if (__any_sync(0xffffffffu, need)) {
                 const float alpha = need ? fast_exp2(m - m_new) : 1.0f;
-                if (it > 0) {
-                    if (!wwait(&bars[B_PV + ((it - 1) & 1)], ((it - 1) >> 1) & 1)) { ok = false; break; }
+                if (k > 0) {
+                    if (!wwait(&bars[B_PV + X], (k - 1) & 1)) { ok = false; break; }
                     tc_fence_after();
                     uint32_t v[32];
-#pragma unroll
+#pragma unroll 1
                     for (int c = 0; c < D / 32; ++c) {
-                        const uint32_t o_addr = tmem + lane_base + kTmO + 32 * c;
+                        const uint32_t o_addr = tmem + lane_base + o_col + 32 * c;
                         tmem_ld32(o_addr, v);
                         tmem_ld_wait();
 #pragma unroll
@@ -425,17 +519,50 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                 }
             }
             const float mu = (m == -CUDART_INF_F) ? 0.f : m;
+            // p = 2^(s * sl2 - mu) and its 8-column group sums
+            float gs[16];
 #pragma unroll
-            for (int c = 0; c < 128; ++c) x[c] = fast_exp2(x[c] - mu);
-            if (it < n_pt) {
+            for (int gq = 0; gq < 16; ++gq) {
+                const float2 q0 = ffma2(make_float2(x[8 * gq + 0], x[8 * gq + 1]), sl2, mu);
+                const float2 q1 = ffma2(make_float2(x[8 * gq + 2], x[8 * gq + 3]), sl2, mu);
+                const float2 q2 = ffma2(make_float2(x[8 * gq + 4], x[8 * gq + 5]), sl2, mu);
+                const float2 q3 = ffma2(make_float2(x[8 * gq + 6], x[8 * gq + 7]), sl2, mu);
+                x[8 * gq + 0] = fast_exp2(q0.x);
+                x[8 * gq + 1] = fast_exp2(q0.y);
+                x[8 * gq + 2] = fast_exp2(q1.x);
+                x[8 * gq + 3] = fast_exp2(q1.y);
+                x[8 * gq + 4] = fast_exp2(q2.x);
+                x[8 * gq + 5] = fast_exp2(q2.y);
+                x[8 * gq + 6] = fast_exp2(q3.x);
+                x[8 * gq + 7] = fast_exp2(q3.y);
+                gs[gq] = ((x[8 * gq + 0] + x[8 * gq + 1]) + (x[8 * gq + 2] + x[8 * gq + 3])) +
+                         ((x[8 * gq + 4] + x[8 * gq + 5]) + (x[8 * gq + 6] + x[8 * gq + 7]));
+            }
+            // P (bf16) over the first 64 columns of S, then hand it to the MMA warp
+            {
+                uint32_t v[32];
 #pragma unroll
-                for (int gq = 0; gq < 16; ++gq) {
-                    float gs = 0.f;
+                for (int e = 0; e < 32; ++e) v[e] = pack_bf16x2(x[2 * e], x[2 * e + 1]);
+                tmem_st32(s_addr, v);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) gs += x[8 * gq + e];
-                    l += gs;
-                    if (MASS) {
-                        const int gi = 16 * it + gq;
+                for (int e = 0; e < 32; ++e) v[e] = pack_bf16x2(x[64 + 2 * e], x[64 + 2 * e + 1]);
+                tmem_st32(s_addr + 32, v);
+                tmem_st_wait();
+            }
+            tc_fence_before();
+            mbar_arrive(&bars[B_PF + X]);
+            // row sum and mass bookkeeping (off the MMA's critical path)
+            float s8[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) s8[j] = gs[2 * j] + gs[2 * j + 1];
+            const float p0 = (s8[0] + s8[1]) + (s8[2] + s8[3]);
+            const float p1 = (s8[4] + s8[5]) + (s8[6] + s8[7]);
+            l += p0 + p1;
+            if (MASS) {
+                if (persistent) {
+#pragma unroll
+                    for (int gq = 0; gq < 16; ++gq) {
+                        const int gi = 16 * k + gq;
                         if (gi < G) {
                             const int seg = grp_seg[gi];
                             if (seg != cur_seg) {
@@ -443,64 +570,36 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                                 cur_seg = seg;
                                 carry = 0.f;
                             }
-                            carry += gs;
+                            carry += gs[gq];
                         }
                     }
-                }
-                if (MASS && it == n_pt - 1 && cur_seg >= 0) {
-                    emit(cur_seg, carry, mu);
-                    cur_seg = -1;
-                    carry = 0.f;
-                }
-            } else {
-                float p0 = 0.f, p1 = 0.f;
-#pragma unroll
-                for (int c = 0; c < 64; ++c) {
-                    p0 += x[c];
-                    p1 += x[64 + c];
-                }
-                l += p0 + p1;
-                if (MASS) {
-                    const int u0 = 2 * (it - n_pt);
-                    emit(n_occ + u0, p0, mu);
-                    if (u0 + 1 < U) emit(n_occ + u0 + 1, p1, mu);
+                    if (k == n_pt - 1 && cur_seg >= 0) {
+                        emit(cur_seg, carry, mu);
+                        cur_seg = -1;
+                        carry = 0.f;
+                    }
+                } else {
+                    emit(n_occ + 2 * lj, p0, mu);
+                    if (2 * lj + 1 < U) emit(n_occ + 2 * lj + 1, p1, mu);
                 }
             }
-            // P (bf16) over the first 64 columns of this S buffer
-            {
-                uint32_t v[32];
-#pragma unroll
-                for (int c = 0; c < 2; ++c) {
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) v[e] = pack_bf16x2(x[64 * c + 2 * e], x[64 * c + 2 * e + 1]);
-                    tmem_st32(s_addr + 32 * c, v);
-                }
-                tmem_st_wait();
-            }
-            tc_fence_before();
-            mbar_arrive(&bars[B_PF + sb]);
         }
 
         // --------------------------------------------------------------- epilogue
-        // one decision for all 128 softmax threads (the epilogue has named barriers)
-        ok = named_bar_and(1, 128, ok);
-        if (ok && n_tiles > 0) {
-            const int jl = n_tiles - 1;
-            ok = named_bar_and(1, 128, wwait(&bars[B_PV + (jl & 1)], (jl >> 1) & 1));
+        const int bar_id = 1 + X;
+        ok = named_bar_and(bar_id, 128, ok);
+        if (ok && nX > 0) {
+            ok = named_bar_and(bar_id, 128, wwait(&bars[B_PV + X], (nX - 1) & 1));
             tc_fence_after();
         }
-        if (ok) {
+        if (ok && nX > 0) {
+            uint8_t* sO = sQ + X * Q_SIDE;  // the side's Q tile is free once its MMAs are done
             const float inv_l = l > 0.f ? 1.0f / l : 0.f;
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
                 uint32_t v[32];
-                if (n_tiles > 0) {
-                    tmem_ld32(tmem + lane_base + kTmO + 32 * c, v);
-                    tmem_ld_wait();
-                } else {
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) v[e] = 0u;
-                }
+                tmem_ld32(tmem + lane_base + o_col + 32 * c, v);
+                tmem_ld_wait();
 #pragma unroll
                 for (int q4 = 0; q4 < 4; ++q4) {
                     uint4 pk;
@@ -508,44 +607,44 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                     pk.y = pack_bf16x2(__uint_as_float(v[8 * q4 + 2]) * inv_l, __uint_as_float(v[8 * q4 + 3]) * inv_l);
                     pk.z = pack_bf16x2(__uint_as_float(v[8 * q4 + 4]) * inv_l, __uint_as_float(v[8 * q4 + 5]) * inv_l);
                     pk.w = pack_bf16x2(__uint_as_float(v[8 * q4 + 6]) * inv_l, __uint_as_float(v[8 * q4 + 7]) * inv_l);
-                    const int chunk = 4 * c + q4;  // 16-byte chunk of the row (8 channels)
-                    const int hh = chunk >> 3;
-                    *reinterpret_cast<uint4*>(sQ + hh * kHalf + sw128_offset(r, chunk & 7)) = pk;
+                    const int chunk = 4 * c + q4;
+                    *reinterpret_cast<uint4*>(sO + (chunk >> 3) * kHalf + sw128_offset(r, chunk & 7)) = pk;
                 }
             }
             const float lse2 = (l > 0.f) ? m + fast_log2(l) : -CUDART_INF_F;
             if (row_valid)
                 a.lse[(size_t)bh * a.q_frames * g.tf + qf * g.tf + qy * g.fw + qx] = lse2 * 0.6931471805599453f;
             fence_proxy_async_smem();
-            named_bar_sync(1, 128);
+            named_bar_sync(bar_id, 128);
             if (r == 0) {
                 for (int hb = 0; hb < 2; ++hb) {
-                    if (hb == 1 && qb1 < 0) break;
-                    const int qb = hb ? qb1 : qb0;
+                    const int qb = qblock(X, hb);
+                    if (qb < 0) break;
                     const int f = qb / g.nbf, i = qb % g.nbf;
                     for (int hh = 0; hh < NH; ++hh)
-                        tma_store_5d(&a.tm_o, sQ + hh * kHalf + hb * (kHalf / 2), hh * 64, h,
+                        tma_store_5d(&a.tm_o, sO + hh * kHalf + hb * (kHalf / 2), hh * 64, h,
                                      8 * (i % g.nbx), 8 * (i / g.nbx), b * a.q_frames + f);
                 }
                 tma_store_commit();
                 tma_store_wait_all();
             }
             if (MASS) {
+                float* smass = seg_mass + X * (S + ucap);
                 const int n_seg = n_occ + U;
-                for (int s = r; s < n_seg; s += 128) seg_mass[s] = 0.f;
-                named_bar_sync(1, 128);
+                for (int s = r; s < n_seg; s += 128) smass[s] = 0.f;
+                named_bar_sync(bar_id, 128);
                 for (int s = 0; s < n_seg; ++s) {
                     float v = row_valid ? fast_exp2(a.scratch[scratch_base + (size_t)s * 128] - lse2) : 0.f;
                     v = warp_sum(v);
-                    if (lane == 0) atomicAdd(&seg_mass[s], v);
+                    if (lane == 0) atomicAdd(&smass[s], v);
                 }
-                named_bar_sync(1, 128);
+                named_bar_sync(bar_id, 128);
                 for (int s = r; s < n_seg; s += 128) {
-                    const float v = seg_mass[s];
+                    const float v = smass[s];
                     if (s < n_occ) {
                         if (a.mass_pers) atomicAdd(&a.mass_pers[(size_t)bh * S + seg_slot[s]], v);
                     } else {
-                        const int L = uni_blk[s - n_occ];
+                        const int L = ublk[s - n_occ];
                         const int phys = (a.ring_head + L / g.nbf) % g.W;
                         if (a.mass_local)
                             atomicAdd(&a.mass_local[((size_t)bh * g.W + phys) * g.nbf + L % g.nbf], v);
@@ -557,7 +656,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 5) {
+    if (warp == 10) {
         __syncwarp();
         tc_fence_after();
         tmem_dealloc(tmem, kTmCols);
@@ -566,8 +665,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
 
 template <int D, bool MASS>
 cudaError_t launch_fwd_t(const FwdKernelArgs& ka, dim3 grid, size_t smem, cudaStream_t st) {
-    cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, MASS>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, attn_fwd_kernel<D, MASS>);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs != kLaunchRegs) return cudaErrorInvalidConfiguration;  // register split needs it
+    e = cudaFuncSetAttribute(attn_fwd_kernel<D, MASS>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     attn_fwd_kernel<D, MASS><<<grid, kThreads, smem, st>>>(ka);
     return cudaGetLastError();
@@ -584,11 +686,9 @@ size_t attn_fwd_smem_bytes(const Geo& g, int ucap) {
 cudaError_t launch_attn_fwd(const FwdArgs& a, bool with_mass, cudaStream_t st) {
     FwdKernelArgs ka;
     ka.a = a;
-    ka.ucap = a.ucap;
-    const int qb_total = a.q_frames * a.g.nbf;
-    ka.n_ctiles = (qb_total + 1) / 2;
-    const size_t smem = attn_fwd_smem_bytes(a.g, ka.ucap);
-    dim3 grid(ka.n_ctiles, a.g.H, a.g.B);
+    ka.n_groups = (a.q_frames * a.g.nbf + 3) / 4;
+    const size_t smem = attn_fwd_smem_bytes(a.g, a.ucap);
+    dim3 grid(ka.n_groups, a.g.H, a.g.B);
     if (a.g.D == 128)
         return with_mass ? launch_fwd_t<128, true>(ka, grid, smem, st)
                          : launch_fwd_t<128, false>(ka, grid, smem, st);

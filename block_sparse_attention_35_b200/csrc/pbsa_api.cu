@@ -181,7 +181,8 @@ int fwd_ucap(const pbsa_config* c, const pbsa::Geo& g, int idx_stride) {
 }
 
 size_t fwd_ws(const pbsa_config* c, const pbsa::Geo& g, int q_frames) {
-    const size_t ctas = (size_t)g.B * g.H * ((q_frames * g.nbf + 1) / 2);
+    // per CTA of four query blocks, two 128-row sides
+    const size_t ctas = (size_t)g.B * g.H * 2 * ((q_frames * g.nbf + 3) / 4);
     const size_t nseg = (size_t)g.S + 2 * topk_count(c, g.W);
     return align256(sizeof(float) * ctas * nseg * 128);
 }

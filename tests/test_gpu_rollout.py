@@ -94,8 +94,11 @@ def test_rollout_twenty_chunks(cuda_dev):
                                       g0, wl.frame_h, wl.frame_w)
                 assert r2["updates"][0][0] == ups, f"step {step}: decision differs at margin {margin}"
             admitted_total += nup
-    # the persistent cache filled up and then kept changing
+    # the persistent cache filled up (chunks 1 and 2 admit 84 blocks each).  Slots keep
+    # accumulating mass while cached, so with stationary synthetic queries later evicted
+    # blocks (two chunks of mass) rank below the slots: every later step checks a merge
+    # that admits nothing, which the decisions above verified against the oracle.
     assert int((a.pers_len > 0).sum().item()) == S
-    assert admitted_total > S
+    assert admitted_total >= S
     print(f"rollout: exact top-k fraction per step {np.round(exact_frac, 3).tolist()}, "
           f"admissions {admitted_total}")
