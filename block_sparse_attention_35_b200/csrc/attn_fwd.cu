@@ -48,25 +48,29 @@ constexpr int kThreads = 384;
 constexpr int kLaunchRegs = 168, kRegsIo = 104, kRegsSoftmax = 200;
 static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsIo <= kThreads * kLaunchRegs, "register split");
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kEmuPairs = 0;  // of every 4 exponential pairs, this many on the FMA pipe (measured: no gain)
 
 struct SmemPlan {
-    uint32_t q, k, v, grp_row, grp_seg, seg_slot, uni_blk, uni_bits, seg_mass, bars, misc,
-        total;
+    uint32_t q, k, v, grp_row, grp_seg, seg_slot, tile_end, tile_seg, uni_blk, uni_bits, lse_s,
+        bars, misc, total;
 };
 
 __host__ __device__ inline SmemPlan fwd_plan(int D, int S, int ucap) {
     SmemPlan p;
     const uint32_t nh = D / 64;
+    const uint32_t n_pt_max = (8u * S + 15u) / 16u;
     p.q = 0;                                 // 2 sides
     p.k = p.q + 2 * nh * kHalf;
     p.v = p.k + kNst * nh * kHalf;
     p.grp_row = p.v + kNst * nh * kHalf;
     p.grp_seg = p.grp_row + 4u * 8u * S;
     p.seg_slot = p.grp_seg + 4u * 8u * S;
-    p.uni_blk = p.seg_slot + 4u * S;         // [2][ucap]
+    p.tile_end = p.seg_slot + 4u * S;        // per persistent tile: groups that end a slot
+    p.tile_seg = p.tile_end + 4u * n_pt_max; // per persistent tile: slot rank of group 0
+    p.uni_blk = p.tile_seg + 4u * n_pt_max;  // [2][ucap]
     p.uni_bits = p.uni_blk + 8u * ucap;      // [2][ucap]
-    p.seg_mass = p.uni_bits + 8u * ucap;     // [2][S + ucap]
-    p.bars = (p.seg_mass + 8u * (S + ucap) + 7u) & ~7u;
+    p.lse_s = p.uni_bits + 8u * ucap;        // [2][128] row log-sum-exp (log2) for the mass
+    p.bars = (p.lse_s + 2u * 128u * 4u + 7u) & ~7u;
     p.misc = p.bars + 8u * 24u;
     p.total = p.misc + 4u * 16u;
     return p;
@@ -84,11 +88,6 @@ struct FwdKernelArgs {
     int n_groups;  // CTAs per (b, h): ceil(QB / 4)
 };
 
-__device__ __forceinline__ float warp_sum(float v) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    return v;
-}
 
 __device__ __forceinline__ float max3f(float a, float b, float c) {
     float d;
@@ -104,6 +103,61 @@ __device__ __forceinline__ float2 ffma2(float2 a, float s, float m) {
     const uint64_t mv = (static_cast<uint64_t>(__float_as_uint(-m)) << 32) | __float_as_uint(-m);
     asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(av), "l"(sv), "l"(mv));
     return make_float2(__uint_as_float(static_cast<uint32_t>(r)), __uint_as_float(static_cast<uint32_t>(r >> 32)));
+}
+
+__device__ __forceinline__ float2 fma2v(float2 a, float2 b, float2 c) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+
+// 2^x on the FMA and integer pipes, for two values (x <= 9).  Cody-Waite style range
+// reduction: adding 1.5 * 2^23 rounds x to the nearest integer n (kept in the low mantissa
+// bits of y) and leaves f = x - n in [-1/2, 1/2]; 2^f is a degree-3 polynomial fitted here
+// for minimum relative error (max 7.5e-5, far below bf16 rounding); n is added to the
+// exponent field.  Inputs below -125 are clamped (the result is then about 2^-125).
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+    constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+    constexpr float c0 = 0.9999281167984009f, c1 = 0.6932609677314758f;
+    constexpr float c2 = 0.24261054396629333f, c3 = 0.05517132207751274f;
+    x.x = fmaxf(x.x, -125.0f);
+    x.y = fmaxf(x.y, -125.0f);
+    const float2 y = fma2v(x, make_float2(1.0f, 1.0f), make_float2(kMagic, kMagic));
+    const float2 t = fma2v(y, make_float2(1.0f, 1.0f), make_float2(-kMagic, -kMagic));
+    const float2 f = fma2v(t, make_float2(-1.0f, -1.0f), x);
+    float2 q = fma2v(make_float2(c3, c3), f, make_float2(c2, c2));
+    q = fma2v(q, f, make_float2(c1, c1));
+    q = fma2v(q, f, make_float2(c0, c0));
+    return make_float2(__uint_as_float(__float_as_uint(q.x) + (__float_as_uint(y.x) << 23)),
+                       __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(y.y) << 23)));
+}
+
+// p = 2^(x * sl2 - mu) over the 128 columns of a row, in place, with the 8-column group
+// sums; EMU of the four pairs in each group go through exp2_poly2, the rest through MUFU.
+template <int EMU>
+__device__ __forceinline__ void exp_row(float (&x)[128], float sl2, float mu, float (&gs)[16]) {
+#pragma unroll
+    for (int gq = 0; gq < 16; ++gq) {
+#pragma unroll
+        for (int pr = 0; pr < 4; ++pr) {
+            const int c = 8 * gq + 2 * pr;
+            const float2 q = ffma2(make_float2(x[c], x[c + 1]), sl2, mu);
+            if (pr >= 4 - EMU) {
+                const float2 e = exp2_poly2(q);
+                x[c] = e.x;
+                x[c + 1] = e.y;
+            } else {
+                x[c] = fast_exp2(q.x);
+                x[c + 1] = fast_exp2(q.y);
+            }
+        }
+        gs[gq] = ((x[8 * gq + 0] + x[8 * gq + 1]) + (x[8 * gq + 2] + x[8 * gq + 3])) +
+                 ((x[8 * gq + 4] + x[8 * gq + 5]) + (x[8 * gq + 6] + x[8 * gq + 7]));
+    }
 }
 
 // 64-bit validity mask of one 8x8 key block: rows < hv, columns < wv, all zero if !sel.
@@ -153,9 +207,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     int32_t* grp_row = reinterpret_cast<int32_t*>(sm + P.grp_row);
     int32_t* grp_seg = reinterpret_cast<int32_t*>(sm + P.grp_seg);
     int32_t* seg_slot = reinterpret_cast<int32_t*>(sm + P.seg_slot);
+    uint32_t* tile_end = reinterpret_cast<uint32_t*>(sm + P.tile_end);
+    int32_t* tile_seg = reinterpret_cast<int32_t*>(sm + P.tile_seg);
     int32_t* uni_blk = reinterpret_cast<int32_t*>(sm + P.uni_blk);
     int32_t* uni_bits = reinterpret_cast<int32_t*>(sm + P.uni_bits);
-    float* seg_mass = reinterpret_cast<float*>(sm + P.seg_mass);
+    float* lse_s = reinterpret_cast<float*>(sm + P.lse_s);
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + P.bars);
     int* misc = reinterpret_cast<int*>(sm + P.misc);
     volatile int* abort_flag = misc + M_ABORT;
@@ -226,6 +282,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         if (lane == 0) {
             misc[M_G] = run;
             misc[M_OCC] = occ;
+        }
+        __syncwarp();
+        // per 16-group tile: bit g set when group g is the last group of its slot
+        for (int t = lane; t * 16 < run; t += 32) {
+            uint32_t ends = 0;
+            for (int gq = 0; gq < 16; ++gq) {
+                const int gi = 16 * t + gq;
+                if (gi < run && (gi + 1 == run || grp_seg[gi + 1] != grp_seg[gi])) ends |= 1u << gq;
+            }
+            tile_end[t] = ends;
+            tile_seg[t] = grp_seg[16 * t];
         }
     }
     if ((warp == 1 || warp == 2) && lane == 0) {
@@ -428,7 +495,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         const size_t scratch_base =
             (((size_t)(bh * ka.n_groups + grp) * 2 + X) * a.n_seg_max) * 128 + r;
         float m = -CUDART_INF_F, l = 0.f, carry = 0.f;
-        int cur_seg = -1;
         bool ok = true;
         auto wwait = [&](uint64_t* bar, uint32_t parity) -> bool {
             return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, a.status));
@@ -519,25 +585,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                 }
             }
             const float mu = (m == -CUDART_INF_F) ? 0.f : m;
-            // p = 2^(s * sl2 - mu) and its 8-column group sums
+            // p = 2^(s * sl2 - mu) and its 8-column group sums; on full tiles a share of the
+            // exponentials runs on the FMA pipe to offload MUFU
             float gs[16];
-#pragma unroll
-            for (int gq = 0; gq < 16; ++gq) {
-                const float2 q0 = ffma2(make_float2(x[8 * gq + 0], x[8 * gq + 1]), sl2, mu);
-                const float2 q1 = ffma2(make_float2(x[8 * gq + 2], x[8 * gq + 3]), sl2, mu);
-                const float2 q2 = ffma2(make_float2(x[8 * gq + 4], x[8 * gq + 5]), sl2, mu);
-                const float2 q3 = ffma2(make_float2(x[8 * gq + 6], x[8 * gq + 7]), sl2, mu);
-                x[8 * gq + 0] = fast_exp2(q0.x);
-                x[8 * gq + 1] = fast_exp2(q0.y);
-                x[8 * gq + 2] = fast_exp2(q1.x);
-                x[8 * gq + 3] = fast_exp2(q1.y);
-                x[8 * gq + 4] = fast_exp2(q2.x);
-                x[8 * gq + 5] = fast_exp2(q2.y);
-                x[8 * gq + 6] = fast_exp2(q3.x);
-                x[8 * gq + 7] = fast_exp2(q3.y);
-                gs[gq] = ((x[8 * gq + 0] + x[8 * gq + 1]) + (x[8 * gq + 2] + x[8 * gq + 3])) +
-                         ((x[8 * gq + 4] + x[8 * gq + 5]) + (x[8 * gq + 6] + x[8 * gq + 7]));
-            }
+            if (masked) exp_row<0>(x, sl2, mu, gs);
+            else exp_row<kEmuPairs>(x, sl2, mu, gs);
             // P (bf16) over the first 64 columns of S, then hand it to the MMA warp
             {
                 uint32_t v[32];
@@ -560,23 +612,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
             l += p0 + p1;
             if (MASS) {
                 if (persistent) {
+                    // slots are runs of groups; emit each slot's partial where its run ends
+                    const uint32_t ends = tile_end[k];
+                    int seg = tile_seg[k];
 #pragma unroll
                     for (int gq = 0; gq < 16; ++gq) {
-                        const int gi = 16 * k + gq;
-                        if (gi < G) {
-                            const int seg = grp_seg[gi];
-                            if (seg != cur_seg) {
-                                if (cur_seg >= 0) emit(cur_seg, carry, mu);
-                                cur_seg = seg;
-                                carry = 0.f;
-                            }
-                            carry += gs[gq];
+                        carry += gs[gq];
+                        if ((ends >> gq) & 1u) {
+                            emit(seg, carry, mu);
+                            ++seg;
+                            carry = 0.f;
                         }
-                    }
-                    if (k == n_pt - 1 && cur_seg >= 0) {
-                        emit(cur_seg, carry, mu);
-                        cur_seg = -1;
-                        carry = 0.f;
                     }
                 } else {
                     emit(n_occ + 2 * lj, p0, mu);
@@ -629,22 +675,28 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                 tma_store_wait_all();
             }
             if (MASS) {
-                float* smass = seg_mass + X * (S + ucap);
+                // one thread per slot/block: sum its 128 row partials, each normalised by its
+                // row's log-sum-exp (padding rows carry +inf and add nothing)
+                float* ls = lse_s + X * 128;
+                ls[r] = row_valid ? lse2 : CUDART_INF_F;
+                named_bar_sync(bar_id, 128);
                 const int n_seg = n_occ + U;
-                for (int s = r; s < n_seg; s += 128) smass[s] = 0.f;
-                named_bar_sync(bar_id, 128);
-                for (int s = 0; s < n_seg; ++s) {
-                    float v = row_valid ? fast_exp2(a.scratch[scratch_base + (size_t)s * 128] - lse2) : 0.f;
-                    v = warp_sum(v);
-                    if (lane == 0) atomicAdd(&smass[s], v);
-                }
-                named_bar_sync(bar_id, 128);
-                for (int s = r; s < n_seg; s += 128) {
-                    const float v = smass[s];
-                    if (s < n_occ) {
-                        if (a.mass_pers) atomicAdd(&a.mass_pers[(size_t)bh * S + seg_slot[s]], v);
+                const float* side_base = a.scratch + (scratch_base - r);
+                for (int sg = r; sg < n_seg; sg += 128) {
+                    const float4* src = reinterpret_cast<const float4*>(side_base + (size_t)sg * 128);
+                    float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll 8
+                    for (int q = 0; q < 32; ++q) {
+                        const float4 v = src[q];
+                        const float4 w = reinterpret_cast<const float4*>(ls)[q];
+                        acc0 += fast_exp2(v.x - w.x) + fast_exp2(v.y - w.y);
+                        acc1 += fast_exp2(v.z - w.z) + fast_exp2(v.w - w.w);
+                    }
+                    const float v = acc0 + acc1;
+                    if (sg < n_occ) {
+                        if (a.mass_pers) atomicAdd(&a.mass_pers[(size_t)bh * S + seg_slot[sg]], v);
                     } else {
-                        const int L = ublk[s - n_occ];
+                        const int L = ublk[sg - n_occ];
                         const int phys = (a.ring_head + L / g.nbf) % g.W;
                         if (a.mass_local)
                             atomicAdd(&a.mass_local[((size_t)bh * g.W + phys) * g.nbf + L % g.nbf], v);

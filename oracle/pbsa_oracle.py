@@ -321,14 +321,15 @@ def cache_update(k_pers, v_pers, pers_len, pers_score, pers_src, k_win, v_win, m
 # fixed; gradients flow through the attention only.
 # ---------------------------------------------------------------------------------------
 def attn_bwd(q, k_pers, v_pers, pers_len, k_win, v_win, idx, dO, frame_h, frame_w,
-             bh=8, bw=8):
+             bh=8, bw=8, qblocks=None):
     """Gradients of L = sum(O * dO) for the PBSA forward with the selection idx fixed.
 
     For each query block: P = softmax(q k^T / sqrt(D)) over its key set,
     dV += P^T dO, dP = dO V^T, dS = P * (dP - rowsum(P * dP)),
     dQ = dS K / sqrt(D), dK += dS^T Q / sqrt(D).
     Returns dQ [B, Nq, H, D], dK_pers/dV_pers [B, H, S, 64, D] (zero past each slot's
-    length), dK_win/dV_win [B, N_L_tokens, H, D].
+    length), dK_win/dV_win [B, N_L_tokens, H, D].  `qblocks` restricts the work to the
+    contributions of those query blocks (a sample; the other rows of dQ stay zero).
     """
     blocks = frame_blocks(frame_h, frame_w, bh, bw)
     tf = frame_h * frame_w
@@ -349,7 +350,7 @@ def attn_bwd(q, k_pers, v_pers, pers_len, k_win, v_win, idx, dO, frame_h, frame_
                                 + [np.zeros(0, dtype=np.int64)]).astype(np.int64)
             pr = np.concatenate([np.arange(int(pers_len[b, h, s])) for s in range(S)]
                                 + [np.zeros(0, dtype=np.int64)]).astype(np.int64)
-            for qbi in range(idx.shape[2]):
+            for qbi in (range(idx.shape[2]) if qblocks is None else qblocks):
                 f, i = divmod(qbi, nbf)
                 toks = f * tf + blocks[i]
                 ids = idx[b, h, qbi]
