@@ -329,7 +329,8 @@ __global__ void __launch_bounds__(kThreads, 1) dkdv_kernel(const __grid_constant
             for (int j = 0; ok && j < n_items; ++j) {
                 const int st = j % kNst;
                 if (!mbar_wait(&qd_full[st], (j / kNst) & 1, abort_flag, a.status)) { ok = false; break; }
-                if (j > 0 && !mbar_wait(pass_done, (j - 1) & 1, abort_flag, a.status)) { ok = false; break; }
+                // no wait for the previous tile's dV/dK MMAs: MMAs issued by this thread run in
+                // issue order, so they finish reading P^T/dS^T before S^T/dP^T overwrite them
                 tc_fence_after();
                 const uint32_t qb_ = smem_u32(sQ + st * TILE), ob = smem_u32(sDO + st * TILE);
 #pragma unroll
@@ -670,7 +671,8 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
                 const int st = it % kNst;
                 if (!mbar_wait(&k_full[st], (it / kNst) & 1, abort_flag, a.status)) { ok = false; break; }
                 if (!mbar_wait(&v_full[st], (it / kNst) & 1, abort_flag, a.status)) { ok = false; break; }
-                if (it > 0 && !mbar_wait(dq_done, (it - 1) & 1, abort_flag, a.status)) { ok = false; break; }
+                // the previous tile's dQ MMAs read dS from TMEM before the next S lands there:
+                // MMAs issued by this thread run in issue order
                 tc_fence_after();
                 const uint32_t kb = smem_u32(sK + st * TILE), vb = smem_u32(sV + st * TILE);
 #pragma unroll
