@@ -11,13 +11,18 @@
 //     persistent slots, or a pair of local blocks); it loops over the query tiles that
 //     attend to those keys (all of them for persistent keys; for local blocks the query
 //     tiles whose query blocks selected either block).  S^T = K Q^T and dP^T = V dO^T land
-//     in TMEM (lanes = keys); each thread owns one key row, forms P^T and dS^T, writes them
-//     as bf16 back over S^T / dP^T, and two TS MMAs accumulate dV += P^T dO and
-//     dK += dS^T Q in TMEM (dO and Q tiles read MN-major from shared memory).
+//     in TMEM (lanes = keys); 16 element warps (a key-row quarter and 32 query columns
+//     each) form P^T and dS^T, write them as bf16 back over S^T / dP^T, and two TS MMAs
+//     accumulate dV += P^T dO and dK += dS^T Q in TMEM (dO and Q tiles read MN-major from
+//     shared memory).
 //  3. dq_kernel: one CTA per query tile (the forward's tiling); per key tile S = Q K^T and
-//     dP = dO V^T in TMEM, each thread (one query row) forms dS, writes it as bf16 over S,
-//     and a TS MMA accumulates dQ += dS K (K read MN-major).
-// Warp roles in 2 and 3: warps 0-3 one row per thread, warp 4 TMA producer, warp 5 MMA.
+//     dP = dO V^T in TMEM, the element warps (a query-row quarter and 32 key columns each)
+//     form dS, write it as bf16 over S, and a TS MMA accumulates dQ += dS K (K read
+//     MN-major).
+// Warp roles in 2 and 3: warps 0-15 elementwise (P, dS), warp 16 TMA producer, warp 17 MMA.
+// The MMA thread issues the next tile's S / dP right after the current tile's gradient
+// MMAs (the tensor pipe runs them in issue order), so only the element warps' work on a
+// tile leaves the pipe idle.
 #include <cuda_bf16.h>
 #include <math_constants.h>
 
@@ -29,7 +34,21 @@ namespace pbsa {
 namespace {
 
 constexpr uint32_t kHalf = 128 * 128;   // 128 rows x 64 bf16 channels
-constexpr int kThreads = 192;
+// Warp roles of the dK/dV and dQ kernels: 16 element warps (four per TMEM lane quarter, each
+// over kCw columns), one TMA producer warp, one MMA warp.
+constexpr int kNwq = 4;
+constexpr int kElemWarps = 4 * kNwq;
+constexpr int kCw = 128 / kNwq;
+constexpr int kProdWarp = kElemWarps;
+constexpr int kMmaWarp = kElemWarps + 1;
+constexpr int kThreads = 32 * (kElemWarps + 2);
+static_assert(kCw == 32, "column masks are 32-bit words");
+
+// TMEM column of the bf16 operand slice kk (16 rows of K) once the element warps have packed
+// their kCw fp32 columns into the first kCw/2 columns of the same range.
+__host__ __device__ constexpr uint32_t packed_col(int kk) {
+    return static_cast<uint32_t>(kCw * (kk / (kCw / 16)) + 8 * (kk % (kCw / 16)));
+}
 constexpr int kNst = 2;
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -177,13 +196,13 @@ __global__ void __launch_bounds__(kThreads, 1) dkdv_kernel(const __grid_constant
             mbar_init(&qd_empty[s], 1);
         }
         mbar_init(sdp_full, 1);
-        mbar_init(pds_full, 128);
+        mbar_init(pds_full, kElemWarps);  // one arrival per element warp
         mbar_init(pass_done, 1);
         mbar_init(drain, 1);
         misc[1] = 0;
         fence_barrier_init();
     }
-    if (warp == 5) tmem_alloc(reinterpret_cast<uint32_t*>(misc + 0), 512);
+    if (warp == kMmaWarp) tmem_alloc(reinterpret_cast<uint32_t*>(misc + 0), 512);
 
     // key set of this CTA
     int G = 0, L0 = -1, L1 = -1;
@@ -247,7 +266,7 @@ __global__ void __launch_bounds__(kThreads, 1) dkdv_kernel(const __grid_constant
     const int n_items = misc[3];
     const bool live = pers_tile ? (tile * 16 < G) : true;
 
-    if (live && warp == 4) {
+    if (live && warp == kProdWarp) {
         // ---------------------------------------------------------- producer
         if (lane == 0) {
             mbar_arrive_expect_tx(kv_full, 2 * TILE);
@@ -319,7 +338,7 @@ __global__ void __launch_bounds__(kThreads, 1) dkdv_kernel(const __grid_constant
             for (int j = max(0, issued - kNst); j < issued; ++j)
                 mbar_wait_drain(&qd_full[j % kNst], (j / kNst) & 1, 100000000ull);
         }
-    } else if (live && warp == 5) {
+    } else if (live && warp == kMmaWarp) {
         // ---------------------------------------------------------------- MMA
         if (lane == 0) {
             constexpr uint32_t id_s = idesc_bf16(128, 128, false, false);
@@ -348,12 +367,12 @@ __global__ void __launch_bounds__(kThreads, 1) dkdv_kernel(const __grid_constant
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
-                    umma_ts(tmem + kTmDV, tmem + kTmS + kk * 8, sdesc_sw128(ob + kk * 2048, kHalf, 1024), id_g,
+                    umma_ts(tmem + kTmDV, tmem + kTmS + packed_col(kk), sdesc_sw128(ob + kk * 2048, kHalf, 1024), id_g,
                             (j > 0 || kk > 0) ? 1u : 0u);
                 }
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
-                    umma_ts(tmem + kTmDK, tmem + kTmP + kk * 8, sdesc_sw128(qb_ + kk * 2048, kHalf, 1024), id_g,
+                    umma_ts(tmem + kTmDK, tmem + kTmP + packed_col(kk), sdesc_sw128(qb_ + kk * 2048, kHalf, 1024), id_g,
                             (j > 0 || kk > 0) ? 1u : 0u);
                 }
                 umma_commit(pass_done);
@@ -364,10 +383,16 @@ __global__ void __launch_bounds__(kThreads, 1) dkdv_kernel(const __grid_constant
                 mbar_wait_drain(drain, 0, 100000000ull);
             }
         }
-    } else if (live) {
-        // ------------------------------------------------- key-row threads (warps 0-3)
-        const int r = threadIdx.x;
-        const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    } else if (live && warp < kElemWarps) {
+        // ------------------------------------------------------- element warps
+        // warp w reads TMEM lanes 32 (w % 4).. (its key rows) and query columns
+        // [32 (w / 4), +32) of S^T / dP^T; it packs P^T / dS^T (bf16) into the first 16 of
+        // those columns once it has read them, so no other warp's input is overwritten.
+        const int wq = warp & 3, cg = warp >> 2;
+        const int r = 32 * wq + lane;
+        const int c0 = kCw * cg;            // first query column of this warp
+        const int hq = c0 >> 6;             // query block (half of the query tile) of those columns
+        const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
         const float sl2 = kLog2e / sqrtf(static_cast<float>(D));
         bool key_valid;
         int kbr = 0;
@@ -393,41 +418,44 @@ __global__ void __launch_bounds__(kThreads, 1) dkdv_kernel(const __grid_constant
             if (!wwait(&qd_full[st], (j / kNst) & 1)) { ok = false; break; }
             if (!wwait(sdp_full, j & 1)) { ok = false; break; }
             tc_fence_after();
-            const int bits = qsel[j];
-            const bool sel0 = key_valid && ((bits >> (2 * kbr + 0)) & 1);
-            const bool sel1 = key_valid && ((bits >> (2 * kbr + 1)) & 1);
-            const float* lse2 = s_lse + st * 128;
-            const float* dl = s_dl + st * 128;
-            uint32_t pk[32], dk[32];
+            const bool sel = key_valid && ((qsel[j] >> (2 * kbr + hq)) & 1);
+            const float4* lse4 = reinterpret_cast<const float4*>(s_lse + st * 128 + c0);
+            const float4* dl4 = reinterpret_cast<const float4*>(s_dl + st * 128 + c0);
+            uint32_t pk[kCw / 2], dk[kCw / 2];
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                uint32_t sv[32], pv[32];
-                tmem_ld32(tmem + lane_base + kTmS + 32 * c, sv);
-                tmem_ld32(tmem + lane_base + kTmP + 32 * c, pv);
+            for (int sc = 0; sc < kCw / 16; ++sc) {
+                uint32_t sv[16], pv[16];
+                tmem_ld16(tmem + lane_base + kTmS + c0 + 16 * sc, sv);
+                tmem_ld16(tmem + lane_base + kTmP + c0 + 16 * sc, pv);
                 tmem_ld_wait();
-                const bool sel = c < 2 ? sel0 : sel1;
 #pragma unroll
-                for (int e = 0; e < 32; e += 2) {
-                    const int q = 32 * c + e;
-                    float p0 = sel ? fast_exp2(__uint_as_float(sv[e]) * sl2 - lse2[q]) : 0.f;
-                    float p1 = sel ? fast_exp2(__uint_as_float(sv[e + 1]) * sl2 - lse2[q + 1]) : 0.f;
-                    const float d0 = p0 * (__uint_as_float(pv[e]) - dl[q]);
-                    const float d1 = p1 * (__uint_as_float(pv[e + 1]) - dl[q + 1]);
-                    pk[16 * (c & 1) + e / 2] = pack_bf16x2(p0, p1);
-                    dk[16 * (c & 1) + e / 2] = pack_bf16x2(d0, d1);
-                }
-                if (c & 1) {
-                    tmem_st32(tmem + lane_base + kTmS + 32 * (c >> 1), pk);
-                    tmem_st32(tmem + lane_base + kTmP + 32 * (c >> 1), dk);
+                for (int e4 = 0; e4 < 4; ++e4) {
+                    const float4 l4 = lse4[4 * sc + e4];
+                    const float4 d4 = dl4[4 * sc + e4];
+                    const float ls[4] = {l4.x, l4.y, l4.z, l4.w};
+                    const float ds[4] = {d4.x, d4.y, d4.z, d4.w};
+                    float p[4], d[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        p[u] = sel ? fast_exp2(__uint_as_float(sv[4 * e4 + u]) * sl2 - ls[u]) : 0.f;
+                        d[u] = p[u] * (__uint_as_float(pv[4 * e4 + u]) - ds[u]);
+                    }
+                    pk[8 * sc + 2 * e4] = pack_bf16x2(p[0], p[1]);
+                    pk[8 * sc + 2 * e4 + 1] = pack_bf16x2(p[2], p[3]);
+                    dk[8 * sc + 2 * e4] = pack_bf16x2(d[0], d[1]);
+                    dk[8 * sc + 2 * e4 + 1] = pack_bf16x2(d[2], d[3]);
                 }
             }
+            tmem_st16(tmem + lane_base + kTmS + c0, pk);
+            tmem_st16(tmem + lane_base + kTmP + c0, dk);
             tmem_st_wait();
             tc_fence_before();
-            mbar_arrive(pds_full);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(pds_full);
         }
-        ok = named_bar_and(1, 128, ok);
+        ok = named_bar_and(2, 32 * kElemWarps, ok);
         if (ok && n_items > 0) {
-            ok = named_bar_and(1, 128, wwait(pass_done, (n_items - 1) & 1));
+            ok = named_bar_and(2, 32 * kElemWarps, wwait(pass_done, (n_items - 1) & 1));
             tc_fence_after();
         }
         if (ok) {
@@ -450,24 +478,24 @@ __global__ void __launch_bounds__(kThreads, 1) dkdv_kernel(const __grid_constant
                 }
             }
             const float isd = 1.0f / sqrtf(static_cast<float>(D));
-#pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-                uint32_t v[32], w[32];
+            // channel chunks of 16: chunk c goes to element warp column group c % kNwq
+            for (int c = cg; c < D / 16; c += kNwq) {
+                uint32_t v[16], w[16];
                 if (n_items > 0) {
-                    tmem_ld32(tmem + lane_base + kTmDV + 32 * c, v);
-                    tmem_ld32(tmem + lane_base + kTmDK + 32 * c, w);
+                    tmem_ld16(tmem + lane_base + kTmDV + 16 * c, v);
+                    tmem_ld16(tmem + lane_base + kTmDK + 16 * c, w);
                     tmem_ld_wait();
                 } else {
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) v[e] = w[e] = 0u;
+                    for (int e = 0; e < 16; ++e) v[e] = w[e] = 0u;
                 }
                 if (key_valid) {
 #pragma unroll
-                    for (int e = 0; e < 32; e += 4) {
-                        *reinterpret_cast<float4*>(dv_row + 32 * c + e) =
+                    for (int e = 0; e < 16; e += 4) {
+                        *reinterpret_cast<float4*>(dv_row + 16 * c + e) =
                             make_float4(__uint_as_float(v[e]), __uint_as_float(v[e + 1]),
                                         __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
-                        *reinterpret_cast<float4*>(dk_row + 32 * c + e) =
+                        *reinterpret_cast<float4*>(dk_row + 16 * c + e) =
                             make_float4(__uint_as_float(w[e]) * isd, __uint_as_float(w[e + 1]) * isd,
                                         __uint_as_float(w[e + 2]) * isd, __uint_as_float(w[e + 3]) * isd);
                     }
@@ -477,7 +505,7 @@ __global__ void __launch_bounds__(kThreads, 1) dkdv_kernel(const __grid_constant
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 5) {
+    if (warp == kMmaWarp) {
         __syncwarp();
         tc_fence_after();
         tmem_dealloc(tmem, 512);
@@ -558,13 +586,13 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
             mbar_init(&kv_empty[s], 1);
         }
         mbar_init(sdp_full, 1);
-        mbar_init(ds_full, 128);
+        mbar_init(ds_full, kElemWarps);
         mbar_init(dq_done, 1);
         mbar_init(drain, 1);
         misc[1] = 0;
         fence_barrier_init();
     }
-    if (warp == 5) tmem_alloc(reinterpret_cast<uint32_t*>(misc + 0), 512);
+    if (warp == kMmaWarp) tmem_alloc(reinterpret_cast<uint32_t*>(misc + 0), 512);
     if (warp == 0) {
         const int G = build_groups(a.pers_len, bh, S, grp_row, a.status);
         if (lane == 0) misc[2] = G;
@@ -608,7 +636,7 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
     const int n_pt = (G + 15) / 16;
     const int n_tiles = n_pt + (U + 1) / 2;
 
-    if (warp == 4) {
+    if (warp == kProdWarp) {
         if (lane == 0) {
             mbar_arrive_expect_tx(q_full, 2 * TILE);
             for (int hb = 0; hb < 2; ++hb) {
@@ -661,7 +689,7 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
                 }
             }
         }
-    } else if (warp == 5) {
+    } else if (warp == kMmaWarp) {
         if (lane == 0) {
             constexpr uint32_t id_s = idesc_bf16(128, 128, false, false);
             constexpr uint32_t id_g = idesc_bf16(128, D, false, true);
@@ -690,7 +718,7 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    umma_ts(tmem + kTmQ, tmem + kTmS + kk * 8, sdesc_sw128(kb + kk * 2048, kHalf, 1024), id_g,
+                    umma_ts(tmem + kTmQ, tmem + kTmS + packed_col(kk), sdesc_sw128(kb + kk * 2048, kHalf, 1024), id_g,
                             (it > 0 || kk > 0) ? 1u : 0u);
                 umma_commit(dq_done);
                 umma_commit(&kv_empty[st]);
@@ -700,8 +728,13 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
                 mbar_wait_drain(drain, 0, 100000000ull);
             }
         }
-    } else {
-        const int r = threadIdx.x;
+    } else if (warp < kElemWarps) {
+        // element warps: warp w owns query rows 32 (w % 4).. (TMEM lanes) and key columns
+        // [32 (w / 4), +32) of S / dP; it packs dS (bf16) into the first 16 of them
+        const int wq = warp & 3, cg = warp >> 2;
+        const int r = 32 * wq + lane;
+        const int c0 = kCw * cg;              // first key column of this warp
+        const int kh = c0 >> 6;               // key block (half of a local key tile) of those columns
         const int hq = r >> 6, rr = r & 63, dy = rr >> 3, dx = rr & 7;
         const int qbr = hq ? qb1 : qb0;
         const int qbv = qbr >= 0 ? qbr : qb0;
@@ -711,7 +744,7 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
         const size_t tok = (size_t)qf * g.tf + qy * g.fw + qx;
         const float lse2 = row_valid ? a.lse[(size_t)bh * nq + tok] * kLog2e : CUDART_INF_F;
         const float dl = row_valid ? a.delta[(size_t)bh * nq + tok] : 0.f;
-        const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+        const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
         const float sl2 = kLog2e / sqrtf(static_cast<float>(D));
         auto wwait = [&](uint64_t* bar, uint32_t parity) -> bool {
             return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, a.status));
@@ -720,78 +753,74 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
         for (int it = 0; it < n_tiles; ++it) {
             if (!wwait(sdp_full, it & 1)) { ok = false; break; }
             tc_fence_after();
-            int nvc = 128;
-            bool sel0 = true, sel1 = true;
-            int hv0 = 8, wv0 = 8, hv1 = 8, wv1 = 8;
-            const bool local = it >= n_pt;
-            if (!local) {
-                nvc = min(128, 8 * (G - 16 * it));
+            // valid-column mask of this warp's 32 key columns
+            uint32_t vmask;
+            if (it < n_pt) {
+                const int nvc = min(128, 8 * (G - 16 * it)) - c0;   // valid persistent columns left
+                vmask = nvc >= kCw ? 0xffffffffu : (nvc <= 0 ? 0u : ((1u << nvc) - 1u));
             } else {
-                const int u0 = 2 * (it - n_pt);
-                const bool has1 = u0 + 1 < U;
-                const int L0 = uni_blk[u0], L1 = has1 ? uni_blk[u0 + 1] : L0;
-                sel0 = (uni_bits[u0] >> hq) & 1;
-                sel1 = has1 && ((uni_bits[u0 + 1] >> hq) & 1);
-                const int i0 = L0 % g.nbf, i1 = L1 % g.nbf;
-                hv0 = min(8, g.fh - 8 * (i0 / g.nbx));
-                wv0 = min(8, g.fw - 8 * (i0 % g.nbx));
-                hv1 = min(8, g.fh - 8 * (i1 / g.nbx));
-                wv1 = min(8, g.fw - 8 * (i1 % g.nbx));
-            }
-            uint32_t dk[32];
+                const int u = 2 * (it - n_pt) + kh;
+                const bool has = u < U;
+                const int L = uni_blk[has ? u : 0];
+                const bool sel = has && ((uni_bits[has ? u : 0] >> hq) & 1);
+                const int i = L % g.nbf;
+                const int hv = min(8, g.fh - 8 * (i / g.nbx)), wv = min(8, g.fw - 8 * (i % g.nbx));
+                // columns c0.. are in-block positions (c0 & 63) + e = 8 y + x
+                const uint32_t rowbits = wv >= 8 ? 0xffu : ((1u << wv) - 1u);
+                uint32_t m = 0;
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                uint32_t sv[32], pv[32];
-                tmem_ld32(tmem + lane_base + kTmS + 32 * c, sv);
-                tmem_ld32(tmem + lane_base + kTmP + 32 * c, pv);
+                for (int yy = 0; yy < kCw / 8; ++yy) {
+                    const int y = ((c0 & 63) >> 3) + yy;
+                    if (y < hv) m |= rowbits << (8 * yy);
+                }
+                vmask = sel ? m : 0u;
+            }
+            uint32_t dk[kCw / 2];
+#pragma unroll
+            for (int sc = 0; sc < kCw / 16; ++sc) {
+                uint32_t sv[16], pv[16];
+                tmem_ld16(tmem + lane_base + kTmS + c0 + 16 * sc, sv);
+                tmem_ld16(tmem + lane_base + kTmP + c0 + 16 * sc, pv);
                 tmem_ld_wait();
 #pragma unroll
-                for (int e = 0; e < 32; e += 2) {
+                for (int e = 0; e < 16; e += 2) {
                     float dsv[2];
 #pragma unroll
                     for (int u = 0; u < 2; ++u) {
-                        const int col = 32 * c + e + u;
-                        bool valid;
-                        if (!local) {
-                            valid = col < nvc;
-                        } else {
-                            const int cc = col & 63;
-                            valid = col < 64 ? (sel0 && (cc >> 3) < hv0 && (cc & 7) < wv0)
-                                             : (sel1 && (cc >> 3) < hv1 && (cc & 7) < wv1);
-                        }
+                        const bool valid = (vmask >> (16 * sc + e + u)) & 1u;
                         const float p = valid ? fast_exp2(__uint_as_float(sv[e + u]) * sl2 - lse2) : 0.f;
                         dsv[u] = p * (__uint_as_float(pv[e + u]) - dl);
                     }
-                    dk[16 * (c & 1) + e / 2] = pack_bf16x2(dsv[0], dsv[1]);
+                    dk[8 * sc + e / 2] = pack_bf16x2(dsv[0], dsv[1]);
                 }
-                if (c & 1) tmem_st32(tmem + lane_base + kTmS + 32 * (c >> 1), dk);
             }
+            tmem_st16(tmem + lane_base + kTmS + c0, dk);
             tmem_st_wait();
             tc_fence_before();
-            mbar_arrive(ds_full);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(ds_full);
         }
-        ok = named_bar_and(1, 128, ok);
+        ok = named_bar_and(2, 32 * kElemWarps, ok);
         if (ok && n_tiles > 0) {
-            ok = named_bar_and(1, 128, wwait(dq_done, (n_tiles - 1) & 1));
+            ok = named_bar_and(2, 32 * kElemWarps, wwait(dq_done, (n_tiles - 1) & 1));
             tc_fence_after();
         }
         if (ok) {
             const float isd = 1.0f / sqrtf(static_cast<float>(D));
             float* dst = a.dq + (((size_t)b * nq + tok) * g.H + h) * D;
-#pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-                uint32_t v[32];
+            for (int c = cg; c < D / 16; c += kNwq) {
+                uint32_t v[16];
                 if (n_tiles > 0) {
-                    tmem_ld32(tmem + lane_base + kTmQ + 32 * c, v);
+                    tmem_ld16(tmem + lane_base + kTmQ + 16 * c, v);
                     tmem_ld_wait();
                 } else {
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) v[e] = 0u;
+                    for (int e = 0; e < 16; ++e) v[e] = 0u;
                 }
                 if (row_valid) {
 #pragma unroll
-                    for (int e = 0; e < 32; e += 4)
-                        *reinterpret_cast<float4*>(dst + 32 * c + e) =
+                    for (int e = 0; e < 16; e += 4)
+                        *reinterpret_cast<float4*>(dst + 16 * c + e) =
                             make_float4(__uint_as_float(v[e]) * isd, __uint_as_float(v[e + 1]) * isd,
                                         __uint_as_float(v[e + 2]) * isd, __uint_as_float(v[e + 3]) * isd);
                 }
@@ -800,7 +829,7 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 5) {
+    if (warp == kMmaWarp) {
         __syncwarp();
         tc_fence_after();
         tmem_dealloc(tmem, 512);
