@@ -355,24 +355,24 @@ __global__ void __launch_bounds__(kThreads, 1) dkdv_kernel(const __grid_constant
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
-                    umma_ss(tmem + kTmS, sdesc_sw128(kb + off, 16, 1024), sdesc_sw128(qb_ + off, 16, 1024), id_s, kk > 0);
+                    umma_ss(tmem + kTmS, sdesc_make(sdesc_lo(kb, 16) + (off >> 4)), sdesc_make(sdesc_lo(qb_, 16) + (off >> 4)), id_s, kk > 0);
                 }
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
-                    umma_ss(tmem + kTmP, sdesc_sw128(vb + off, 16, 1024), sdesc_sw128(ob + off, 16, 1024), id_s, kk > 0);
+                    umma_ss(tmem + kTmP, sdesc_make(sdesc_lo(vb, 16) + (off >> 4)), sdesc_make(sdesc_lo(ob, 16) + (off >> 4)), id_s, kk > 0);
                 }
                 umma_commit(sdp_full);
                 if (!mbar_wait(pds_full, j & 1, abort_flag, a.status)) { ok = false; break; }
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
-                    umma_ts(tmem + kTmDV, tmem + kTmS + packed_col(kk), sdesc_sw128(ob + kk * 2048, kHalf, 1024), id_g,
+                    umma_ts(tmem + kTmDV, tmem + kTmS + packed_col(kk), sdesc_make(sdesc_lo(ob, kHalf) + kk * 128), id_g,
                             (j > 0 || kk > 0) ? 1u : 0u);
                 }
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
-                    umma_ts(tmem + kTmDK, tmem + kTmP + packed_col(kk), sdesc_sw128(qb_ + kk * 2048, kHalf, 1024), id_g,
+                    umma_ts(tmem + kTmDK, tmem + kTmP + packed_col(kk), sdesc_make(sdesc_lo(qb_, kHalf) + kk * 128), id_g,
                             (j > 0 || kk > 0) ? 1u : 0u);
                 }
                 umma_commit(pass_done);
@@ -706,19 +706,19 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
-                    umma_ss(tmem + kTmS, sdesc_sw128(qbase + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024), id_s, kk > 0);
+                    umma_ss(tmem + kTmS, sdesc_make(sdesc_lo(qbase, 16) + (off >> 4)), sdesc_make(sdesc_lo(kb, 16) + (off >> 4)), id_s, kk > 0);
                 }
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
-                    umma_ss(tmem + kTmP, sdesc_sw128(obase + off, 16, 1024), sdesc_sw128(vb + off, 16, 1024), id_s, kk > 0);
+                    umma_ss(tmem + kTmP, sdesc_make(sdesc_lo(obase, 16) + (off >> 4)), sdesc_make(sdesc_lo(vb, 16) + (off >> 4)), id_s, kk > 0);
                 }
                 umma_commit(sdp_full);
                 if (!mbar_wait(ds_full, it & 1, abort_flag, a.status)) { ok = false; break; }
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    umma_ts(tmem + kTmQ, tmem + kTmS + packed_col(kk), sdesc_sw128(kb + kk * 2048, kHalf, 1024), id_g,
+                    umma_ts(tmem + kTmQ, tmem + kTmS + packed_col(kk), sdesc_make(sdesc_lo(kb, kHalf) + kk * 128), id_g,
                             (it > 0 || kk > 0) ? 1u : 0u);
                 umma_commit(dq_done);
                 umma_commit(&kv_empty[st]);

@@ -136,12 +136,13 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
                        __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(y.y) << 23)));
 }
 
-// p = 2^(x * sl2 - mu) over the 128 columns of a row, in place, with the 8-column group
-// sums; EMU of the four pairs in each group go through exp2_poly2, the rest through MUFU.
-template <int EMU>
-__device__ __forceinline__ void exp_row(float (&x)[128], float sl2, float mu, float (&gs)[16]) {
+// p = 2^(x * sl2 - mu) over the 64 columns [64 H, 64 H + 64) of a row, in place, with their
+// 8-column group sums; EMU of the four pairs in each group go through exp2_poly2, the rest
+// through MUFU.
+template <int EMU, int H>
+__device__ __forceinline__ void exp_half(float (&x)[128], float sl2, float mu, float (&gs)[16]) {
 #pragma unroll
-    for (int gq = 0; gq < 16; ++gq) {
+    for (int gq = 8 * H; gq < 8 * H + 8; ++gq) {
 #pragma unroll
         for (int pr = 0; pr < 4; ++pr) {
             const int c = 8 * gq + 2 * pr;
@@ -426,7 +427,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                 const uint32_t v_base = smem_u32(sV + st * KV_BYTES);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    umma_ts(o_tmem, p_tmem + kk * 8, sdesc_sw128(v_base + kk * 2048, kHalf, 1024), idesc_pv,
+                    umma_ts(o_tmem, p_tmem + kk * 8, sdesc_make(sdesc_lo(v_base, kHalf) + kk * 128), idesc_pv,
                             (npv[X] > 0 || kk > 0) ? 1u : 0u);
                 umma_commit(&bars[B_PV + X]);
                 ++npv[X];
@@ -449,7 +450,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
 #pragma unroll
                         for (int kk = 0; kk < D / 16; ++kk) {
                             const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
-                            umma_ss(s_tmem, sdesc_sw128(q_base + off, 16, 1024), sdesc_sw128(k_base + off, 16, 1024),
+                            umma_ss(s_tmem, sdesc_make(sdesc_lo(q_base, 16) + (off >> 4)), sdesc_make(sdesc_lo(k_base, 16) + (off >> 4)),
                                     idesc_qk, kk > 0 ? 1u : 0u);
                         }
                         umma_commit(&bars[B_SF + X]);
@@ -541,6 +542,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                 mk1 = block_mask(sel1, min(8, g.fh - 8 * (i1 / g.nbx)), min(8, g.fw - 8 * (i1 % g.nbx)));
                 masked = true;
             }
+            masked = masked && (mk0 != ~0ull || mk1 != ~0ull);
             if (masked) {
 #pragma unroll
                 for (int c = 0; c < 64; ++c) {
@@ -585,20 +587,23 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                 }
             }
             const float mu = (m == -CUDART_INF_F) ? 0.f : m;
-            // p = 2^(s * sl2 - mu) and its 8-column group sums; on full tiles a share of the
-            // exponentials runs on the FMA pipe to offload MUFU
+            // p = 2^(s * sl2 - mu) and its 8-column group sums, one half of the row at a time;
+            // each half's P (bf16) goes over the first 64 columns of S as soon as it is done, so
+            // the first store overlaps the second half's exponentials.  On unmasked tiles a
+            // share of the exponentials runs on the FMA pipe to offload MUFU.
             float gs[16];
-            if (masked) exp_row<0>(x, sl2, mu, gs);
-            else exp_row<kEmuPairs>(x, sl2, mu, gs);
-            // P (bf16) over the first 64 columns of S, then hand it to the MMA warp
             {
-                uint32_t v[32];
+                uint32_t v0[32], v1[32];
+                if (masked) exp_half<0, 0>(x, sl2, mu, gs);
+                else exp_half<kEmuPairs, 0>(x, sl2, mu, gs);
 #pragma unroll
-                for (int e = 0; e < 32; ++e) v[e] = pack_bf16x2(x[2 * e], x[2 * e + 1]);
-                tmem_st32(s_addr, v);
+                for (int e = 0; e < 32; ++e) v0[e] = pack_bf16x2(x[2 * e], x[2 * e + 1]);
+                tmem_st32(s_addr, v0);
+                if (masked) exp_half<0, 1>(x, sl2, mu, gs);
+                else exp_half<kEmuPairs, 1>(x, sl2, mu, gs);
 #pragma unroll
-                for (int e = 0; e < 32; ++e) v[e] = pack_bf16x2(x[64 + 2 * e], x[64 + 2 * e + 1]);
-                tmem_st32(s_addr + 32, v);
+                for (int e = 0; e < 32; ++e) v1[e] = pack_bf16x2(x[64 + 2 * e], x[64 + 2 * e + 1]);
+                tmem_st32(s_addr + 32, v1);
                 tmem_st_wait();
             }
             tc_fence_before();

@@ -170,6 +170,17 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
     return d;
 }
 
+// The same descriptor split in two: the low word (start address and leading byte offset)
+// changes per operand slice, the high word (SBO = 1024, version, 128B swizzle) never does, so
+// an MMA loop adds a constant (offset >> 4) to one precomputed low word per slice.
+__device__ __forceinline__ uint32_t sdesc_lo(uint32_t saddr, uint32_t lbo) {
+    return ((saddr >> 4) & 0x3FFFu) | (((lbo >> 4) & 0x3FFFu) << 16);
+}
+constexpr uint32_t kSdescHi = ((1024u >> 4) & 0x3FFFu) | (1u << 14) | (2u << 29);
+__device__ __forceinline__ uint64_t sdesc_make(uint32_t lo) {
+    return (static_cast<uint64_t>(kSdescHi) << 32) | lo;
+}
+
 // Instruction descriptor of kind::f16 with bf16 A/B and fp32 accumulate.
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn_major, bool b_mn_major) {
     return (1u << 4)                               // D format: f32
