@@ -271,13 +271,8 @@ __global__ void __launch_bounds__(kThreads, 1) dkdv_kernel(const __grid_constant
         if (lane == 0) {
             mbar_arrive_expect_tx(kv_full, 2 * TILE);
             if (pers_tile) {
-                for (int c = 0; c < 16; ++c) {
-                    const int row = grp_row[min(tile * 16 + c, G - 1)];
-                    for (int hh = 0; hh < NH; ++hh) {
-                        tma_load_2d(sK + hh * kHalf + c * 1024, &a.tm_kp, kv_full, hh * 64, row);
-                        tma_load_2d(sV + hh * kHalf + c * 1024, &a.tm_vp, kv_full, hh * 64, row);
-                    }
-                }
+                tma_load_groups16<NH>(sK, kHalf, &a.tm_kp, &a.tm_kp64, grp_row, tile * 16, G, kv_full);
+                tma_load_groups16<NH>(sV, kHalf, &a.tm_vp, &a.tm_vp64, grp_row, tile * 16, G, kv_full);
             } else {
                 for (int kb = 0; kb < 2; ++kb) {
                     const int L = (kb == 1 && L1 >= 0) ? L1 : L0;

@@ -352,11 +352,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         if (lane == 0) {
             const bool isK = warp == 8;
             const CUtensorMap* mp = isK ? &a.tm_kp : &a.tm_vp;
+            const CUtensorMap* mp64 = isK ? &a.tm_kp64 : &a.tm_vp64;
             const CUtensorMap* ml = isK ? &a.tm_kl : &a.tm_vl;
             uint8_t* base = isK ? sK : sV;
             uint64_t* full = &bars[isK ? B_KF : B_VF];
             uint64_t* empty = &bars[isK ? B_KE : B_VE];
             tma_prefetch_desc(mp);
+            tma_prefetch_desc(mp64);
             tma_prefetch_desc(ml);
             if (isK) {
                 tma_prefetch_desc(&a.tm_q);
@@ -380,11 +382,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                 int lj;
                 const int cons = tile_cons(t, n_pt, nla, nlb, has_b, &lj);
                 if (lj < 0) {
-                    for (int c = 0; c < 16; ++c) {
-                        const int row = grp_row[min(t * 16 + c, G - 1)];
-                        for (int hh = 0; hh < NH; ++hh)
-                            tma_load_2d(dst + hh * kHalf + c * 1024, mp, &full[st], hh * 64, row);
-                    }
+                    tma_load_groups16<NH>(dst, kHalf, mp, mp64, grp_row, t * 16, G, &full[st]);
                 } else {
                     const int X = cons == 2 ? 1 : 0;
                     const int U = X ? UB : UA;

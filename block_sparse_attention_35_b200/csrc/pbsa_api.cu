@@ -156,12 +156,12 @@ int map_tokens(CUtensorMap* m, const void* ptr, const pbsa::Geo& g, long long fr
 }
 
 // [rows, D] bf16 tensor (persistent slots, 64 rows each), box [8, 64], 128-byte swizzle.
-int map_rows(CUtensorMap* m, const void* ptr, const pbsa::Geo& g, long long rows) {
+int map_rows(CUtensorMap* m, const void* ptr, const pbsa::Geo& g, long long rows, int box_rows = 8) {
     auto enc = encode_fn();
     if (!enc) return fail(PBSA_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
     cuuint64_t dims[2] = {(cuuint64_t)g.D, (cuuint64_t)rows};
     cuuint64_t strides[1] = {(cuuint64_t)g.D * 2};
-    cuuint32_t box[2] = {64, 8};
+    cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
     cuuint32_t es[2] = {1, 1};
     CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, es,
                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -323,6 +323,8 @@ int pbsa_attn_fwd(const pbsa_config* cfg, const void* q, int q_frames, const voi
     if ((rc = map_tokens(&a.tm_vl, v_local, g, (long long)g.B * g.W)) != PBSA_OK) return rc;
     if ((rc = map_rows(&a.tm_kp, k_pers, g, (long long)g.B * g.H * g.S * 64)) != PBSA_OK) return rc;
     if ((rc = map_rows(&a.tm_vp, v_pers, g, (long long)g.B * g.H * g.S * 64)) != PBSA_OK) return rc;
+    if ((rc = map_rows(&a.tm_kp64, k_pers, g, (long long)g.B * g.H * g.S * 64, 64)) != PBSA_OK) return rc;
+    if ((rc = map_rows(&a.tm_vp64, v_pers, g, (long long)g.B * g.H * g.S * 64, 64)) != PBSA_OK) return rc;
     cudaError_t e = pbsa::launch_attn_fwd(a, with_mass, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "forward kernel launch");
     return PBSA_OK;
@@ -387,6 +389,8 @@ int pbsa_attn_bwd(const pbsa_config* cfg, const void* q, int q_frames, const voi
     if ((rc = map_tokens(&a.tm_vl, v_local, g, (long long)g.B * g.W)) != PBSA_OK) return rc;
     if ((rc = map_rows(&a.tm_kp, k_pers, g, (long long)g.B * g.H * g.S * 64)) != PBSA_OK) return rc;
     if ((rc = map_rows(&a.tm_vp, v_pers, g, (long long)g.B * g.H * g.S * 64)) != PBSA_OK) return rc;
+    if ((rc = map_rows(&a.tm_kp64, k_pers, g, (long long)g.B * g.H * g.S * 64, 64)) != PBSA_OK) return rc;
+    if ((rc = map_rows(&a.tm_vp64, v_pers, g, (long long)g.B * g.H * g.S * 64, 64)) != PBSA_OK) return rc;
     cudaError_t e = pbsa::launch_attn_bwd(a, static_cast<cudaStream_t>(stream));
     if (e == cudaErrorNotSupported) return fail(PBSA_ERR_UNSUPPORTED, "backward kernel not built");
     if (e != cudaSuccess) return cuda_fail(e, "backward kernel launch");

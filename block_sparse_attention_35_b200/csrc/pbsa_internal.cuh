@@ -36,6 +36,7 @@ struct FwdArgs {
     float* scratch;      // mass partials, [ctas][n_seg_max][128]
     int32_t* status;
     CUtensorMap tm_q, tm_o, tm_kl, tm_vl, tm_kp, tm_vp;
+    CUtensorMap tm_kp64, tm_vp64;  // slot store, 64-row boxes (one full slot)
 };
 
 // Backward-pass launch arguments.
@@ -58,6 +59,7 @@ struct BwdArgs {
     float* dv_local;
     int32_t* status;
     CUtensorMap tm_q, tm_do, tm_kl, tm_vl, tm_kp, tm_vp;
+    CUtensorMap tm_kp64, tm_vp64;
 };
 
 // Launchers (return a cudaError_t from the launch).
