@@ -49,6 +49,7 @@ def parse():
     ap.add_argument("--no-bwd", action="store_true", help="time select/fwd/slide only")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    ap.add_argument("--no-dense", action="store_true", help="skip the dense-attention comparison")
     return ap.parse_args()
 
 
@@ -363,6 +364,9 @@ def run_ours(args, ws, rank, local):
         cpu = {"value": fl / dt / 1e12, "unit": UNIT, "cores": threads, "kind": "oracle",
                "sample": f"2 of 12 heads of the decode chunk: select + forward with mass + "
                          f"backward + merge ({dt:.1f} s)"}
+    dense = None
+    if rank == 0 and not args.no_dense:
+        dense = run_dense(dev, sets[0])
     if rank == 0:
         out = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
@@ -379,12 +383,76 @@ def run_ours(args, ws, rank, local):
                          "achieved": dominant["achieved"], "peak": peak_tf, "unit": "TFLOP/s",
                          "frac": dominant["achieved"] / peak_tf, "traffic": traffic,
                          "peak_source": f"{peak_src} bf16 burst"},
+            "roofline_fwd": {"bound": "tensor", "kernel": "attn_fwd (with block mass)",
+                             "achieved": fwd_ach, "peak": peak_tf, "unit": "TFLOP/s",
+                             "frac": fwd_ach / peak_tf, "ms": fwd_avg},
+            "dense": dense,
             "cpu_baseline": cpu,
             "clocks": ck,
             "e2e": e2e,
             "gpu_launches": kernels_per_step(with_bwd) * args.steps,
         }
         print(json.dumps(out))
+
+
+def _time_ms(fn, reps=10, warm=3):
+    for _ in range(warm):
+        fn()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    t0.record()
+    for _ in range(reps):
+        fn()
+    t1.record()
+    torch.cuda.synchronize()
+    return t0.elapsed_time(t1) / reps
+
+
+def run_dense(dev, first_set):
+    """The dense comparison at the same shapes on the same GPU: torch's scaled-dot-product
+    attention (bf16, its flash kernel) over the whole cache (every persistent slot row and
+    every window token, 18720 keys), the PBSA forward at ratio 1 (every local block
+    selected), and the PBSA forward at the workload's ratio, the last two without block
+    mass.  Warm L2, 10 launches each."""
+    from block_sparse_attention_35_b200.attention import SparseForcingAttention
+    a, q, _ = first_set
+    nq = q.shape[1]
+    qd = q.permute(0, 2, 1, 3).contiguous()                               # [B, H, Nq, D]
+    kp = a.k_pers.reshape(WL.B, WL.H, -1, WL.D)                            # [B, H, S*64, D]
+    kd = torch.cat([kp, a.k_local.permute(0, 2, 1, 3)], dim=2).contiguous()
+    vp = a.v_pers.reshape(WL.B, WL.H, -1, WL.D)
+    vd = torch.cat([vp, a.v_local.permute(0, 2, 1, 3)], dim=2).contiguous()
+    nk = kd.shape[2]
+    sdpa = torch.nn.functional.scaled_dot_product_attention
+    sdpa_ms = _time_ms(lambda: sdpa(qd, kd, vd))
+    qg = qd.clone().requires_grad_(True)
+    kg = kd.clone().requires_grad_(True)
+    vg = vd.clone().requires_grad_(True)
+    go = torch.randn_like(qd)
+
+    def fb():
+        o = sdpa(qg, kg, vg)
+        o.backward(go)
+    sdpa_fb_ms = _time_ms(fb)
+    a.select(q)
+    pbsa_ms = _time_ms(lambda: a.attend(q, accumulate_mass=False))
+    a1 = SparseForcingAttention(WL.B, WL.H, WL.D, WL.frame_h, WL.frame_w, WL.total_cache_size,
+                                WL.local_cache_size, WL.persistent_cache_size,
+                                max_seq_len=WL.max_seq_len, local_block_sparse_topk_ratio=1.0,
+                                chunk_frames=WL.q_frames, device=dev)
+    a1.k_local.copy_(a.k_local)
+    a1.v_local.copy_(a.v_local)
+    a1.local_frames = a1.W
+    a1.load_persistent(a.k_pers, a.v_pers, a.pers_len)
+    a1.select(q)
+    ratio1_ms = _time_ms(lambda: a1.attend(q, accumulate_mass=False))
+    dense_fl = 4.0 * WL.D * nq * nk * WL.H
+    return {"sdpa_fwd_ms": sdpa_ms, "sdpa_fwd_bwd_ms": sdpa_fb_ms,
+            "sdpa_fwd_tflops": dense_fl / (sdpa_ms * 1e-3) / 1e12,
+            "pbsa_fwd_ms": pbsa_ms, "pbsa_ratio1_fwd_ms": ratio1_ms,
+            "keys_dense": nk, "note": "forward without block mass; warm L2; sdpa keys include "
+                                      "the persistent slots' padding rows"}
 
 
 def run_e2e(args, sets, dev, with_bwd, fwd_flops, bwd_flops, ws):
