@@ -136,6 +136,31 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
                        __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(y.y) << 23)));
 }
 
+// exp_half<0, 0> plus the maximum of all 128 raw values, read before they are overwritten:
+// the ALU max work interleaves with the MUFU exponentials.
+__device__ __forceinline__ float exp_half0_max(float (&x)[128], float sl2, float mu, float (&gs)[16]) {
+    float mx[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) mx[j] = -CUDART_INF_F;
+#pragma unroll
+    for (int gq = 0; gq < 8; ++gq) {
+#pragma unroll
+        for (int j = 0; j < 8; j += 2) mx[j / 2] = max3f(mx[j / 2], x[8 * gq + j], x[8 * gq + j + 1]);
+#pragma unroll
+        for (int j = 0; j < 8; j += 2) mx[4 + j / 2] = max3f(mx[4 + j / 2], x[64 + 8 * gq + j], x[64 + 8 * gq + j + 1]);
+#pragma unroll
+        for (int pr = 0; pr < 4; ++pr) {
+            const int c = 8 * gq + 2 * pr;
+            const float2 q = ffma2(make_float2(x[c], x[c + 1]), sl2, mu);
+            x[c] = fast_exp2(q.x);
+            x[c + 1] = fast_exp2(q.y);
+        }
+        gs[gq] = ((x[8 * gq + 0] + x[8 * gq + 1]) + (x[8 * gq + 2] + x[8 * gq + 3])) +
+                 ((x[8 * gq + 4] + x[8 * gq + 5]) + (x[8 * gq + 6] + x[8 * gq + 7]));
+    }
+    return max3f(max3f(mx[0], mx[1], mx[2]), max3f(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
+}
+
 // p = 2^(x * sl2 - mu) over the 64 columns [64 H, 64 H + 64) of a row, in place, with their
 // 8-column group sums; EMU of the four pairs in each group go through exp2_poly2, the rest
 // through MUFU.
@@ -507,7 +532,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
             tc_fence_after();
             const uint32_t s_addr = tmem + lane_base + s_col;
             float x[128];
-            {
+            auto load_s = [&]() {
                 uint32_t v[4][32];
 #pragma unroll
                 for (int c = 0; c < 4; ++c) tmem_ld32(s_addr + 32 * c, v[c]);
@@ -516,7 +541,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                 for (int c = 0; c < 4; ++c)
 #pragma unroll
                     for (int e = 0; e < 32; ++e) x[32 * c + e] = __uint_as_float(v[c][e]);
-            }
+            };
+            load_s();
             const bool persistent = k < n_pt;
             int lj = 0;
             bool masked;
@@ -541,24 +567,22 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                 masked = true;
             }
             masked = masked && (mk0 != ~0ull || mk1 != ~0ull);
-            if (masked) {
+            auto apply_mask = [&]() {
 #pragma unroll
                 for (int c = 0; c < 64; ++c) {
                     if (!((mk0 >> c) & 1ull)) x[c] = -CUDART_INF_F;
                     if (!((mk1 >> c) & 1ull)) x[64 + c] = -CUDART_INF_F;
                 }
-            }
-            // row maximum of the raw scores (tree of 3-input max)
-            float mx[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) mx[j] = x[j];
-#pragma unroll
-            for (int c = 8; c + 16 <= 128; c += 16)
-#pragma unroll
-                for (int j = 0; j < 8; ++j) mx[j] = max3f(mx[j], x[c + j], x[c + 8 + j]);
-            float mt = max3f(max3f(mx[0], mx[1], mx[2]), max3f(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
-#pragma unroll
-            for (int c = 120; c < 128; ++c) mt = fmaxf(mt, x[c]);
+            };
+            if (masked) apply_mask();
+            // Optimistic pass: the first half's exponentials against the running reference m
+            // (what the lazy rescale uses whenever no row's maximum grew by more than 2^8),
+            // with the tile's row maximum taken in the same pass.  Only when some row of the
+            // warp needs a new reference (and always on the first tile) does the warp rescale
+            // O and l, reload S from TMEM (still intact: nothing is stored yet) and redo the
+            // first half.
+            float gs[16];
+            const float mt = exp_half0_max(x, sl2, (m == -CUDART_INF_F) ? 0.f : m, gs);
             const float m_new = fmaxf(m, mt * sl2);
             const bool need = m_new > m + 8.0f;
             if (__any_sync(0xffffffffu, need)) {
@@ -583,17 +607,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                     carry *= alpha;
                     m = m_new;
                 }
+                load_s();
+                if (masked) apply_mask();
+                exp_half<0, 0>(x, sl2, (m == -CUDART_INF_F) ? 0.f : m, gs);
             }
             const float mu = (m == -CUDART_INF_F) ? 0.f : m;
-            // p = 2^(s * sl2 - mu) and its 8-column group sums, one half of the row at a time;
             // each half's P (bf16) goes over the first 64 columns of S as soon as it is done, so
-            // the first store overlaps the second half's exponentials.  On unmasked tiles a
-            // share of the exponentials runs on the FMA pipe to offload MUFU.
-            float gs[16];
+            // the first store overlaps the second half's exponentials
             {
                 uint32_t v0[32], v1[32];
-                if (masked) exp_half<0, 0>(x, sl2, mu, gs);
-                else exp_half<kEmuPairs, 0>(x, sl2, mu, gs);
 #pragma unroll
                 for (int e = 0; e < 32; ++e) v0[e] = pack_bf16x2(x[2 * e], x[2 * e + 1]);
                 tmem_st32(s_addr, v0);
