@@ -138,6 +138,7 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
 
 // exp_half<0, 0> plus the maximum of all 128 raw values, read before they are overwritten:
 // the ALU max work interleaves with the MUFU exponentials.
+template <int EMU>
 __device__ __forceinline__ float exp_half0_max(float (&x)[128], float sl2, float mu, float (&gs)[16]) {
     float mx[8];
 #pragma unroll
@@ -152,8 +153,14 @@ __device__ __forceinline__ float exp_half0_max(float (&x)[128], float sl2, float
         for (int pr = 0; pr < 4; ++pr) {
             const int c = 8 * gq + 2 * pr;
             const float2 q = ffma2(make_float2(x[c], x[c + 1]), sl2, mu);
-            x[c] = fast_exp2(q.x);
-            x[c + 1] = fast_exp2(q.y);
+            if (pr >= 4 - EMU) {
+                const float2 e = exp2_poly2(q);
+                x[c] = e.x;
+                x[c + 1] = e.y;
+            } else {
+                x[c] = fast_exp2(q.x);
+                x[c + 1] = fast_exp2(q.y);
+            }
         }
         gs[gq] = ((x[8 * gq + 0] + x[8 * gq + 1]) + (x[8 * gq + 2] + x[8 * gq + 3])) +
                  ((x[8 * gq + 4] + x[8 * gq + 5]) + (x[8 * gq + 6] + x[8 * gq + 7]));
@@ -582,7 +589,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
             // O and l, reload S from TMEM (still intact: nothing is stored yet) and redo the
             // first half.
             float gs[16];
-            const float mt = exp_half0_max(x, sl2, (m == -CUDART_INF_F) ? 0.f : m, gs);
+            const float mu0 = (m == -CUDART_INF_F) ? 0.f : m;
+            const float mt = masked ? exp_half0_max<0>(x, sl2, mu0, gs) : exp_half0_max<kEmuPairs>(x, sl2, mu0, gs);
             const float m_new = fmaxf(m, mt * sl2);
             const bool need = m_new > m + 8.0f;
             if (__any_sync(0xffffffffu, need)) {
