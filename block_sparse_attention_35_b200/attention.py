@@ -27,6 +27,8 @@ class SparseForcingAttention:
                  use_local_block_sparse_attn: bool = True,
                  local_block_sparse_topk_ratio: float = 0.125, chunk_frames: int = 3,
                  device="cuda"):
+        # kv_cache_mode="dense": one window of total_cache_size tokens, no persistent slots
+        # (S = 0), every block attended; slide() then only drops the oldest frames
         self.cfg = P.make_config(B, H, D, frame_h, frame_w, total_cache_size, local_cache_size,
                                  persistent_cache_size, max_seq_len,
                                  local_block_sparse_topk_ratio, use_local_block_sparse_attn,

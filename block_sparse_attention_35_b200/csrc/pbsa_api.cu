@@ -40,7 +40,13 @@ int blocks_per_frame(const pbsa_config* c) {
     return ((c->frame_h + 7) / 8) * ((c->frame_w + 7) / 8);
 }
 
+bool dense_mode(const pbsa_config* c) { return c->kv_cache_mode == PBSA_KV_CACHE_DENSE; }
+
+// tokens of the local ring: the local cache, or the whole cache in dense mode
+int window_tokens(const pbsa_config* c) { return dense_mode(c) ? c->total_cache_size : c->local_cache_size; }
+
 int num_slots(const pbsa_config* c) {
+    if (dense_mode(c)) return 0;
     const int tf = tokens_per_frame(c);
     if (c->persistent_cache_size % tf == 0) return c->persistent_cache_size / tf * blocks_per_frame(c);
     return (c->persistent_cache_size + 63) / 64;
@@ -49,7 +55,7 @@ int num_slots(const pbsa_config* c) {
 int topk_count(const pbsa_config* c, int local_frames) {
     const int nl = local_frames * blocks_per_frame(c);
     if (nl <= 0) return 0;
-    if (!c->use_local_block_sparse_attn) return nl;
+    if (!c->use_local_block_sparse_attn || dense_mode(c)) return nl;
     const double k = std::ceil(static_cast<double>(c->local_block_sparse_topk_ratio) * nl);
     int ki = static_cast<int>(k);
     if (ki < 1) ki = 1;
@@ -67,12 +73,16 @@ int validate(const pbsa_config* c) {
     if (c->block_t != 1 || c->block_h != 8 || c->block_w != 8)
         return fail(PBSA_ERR_UNSUPPORTED, "sparse_kv_block_size [%d,%d,%d]: only [1,8,8] is built",
                     c->block_t, c->block_h, c->block_w);
-    if (c->kv_cache_mode != PBSA_KV_CACHE_SPARSE_FORCING)
-        return fail(PBSA_ERR_UNSUPPORTED, "kv_cache_mode %d: only sparse_forcing is built", c->kv_cache_mode);
+    if (c->kv_cache_mode != PBSA_KV_CACHE_SPARSE_FORCING && c->kv_cache_mode != PBSA_KV_CACHE_DENSE)
+        return fail(PBSA_ERR_UNSUPPORTED, "kv_cache_mode %d: only sparse_forcing and dense are built",
+                    c->kv_cache_mode);
     const int tf = tokens_per_frame(c);
     if (c->local_cache_size < tf || c->local_cache_size % tf)
         return fail(PBSA_ERR_ARG, "local_cache_size %d is not a positive multiple of %d tokens/frame",
                     c->local_cache_size, tf);
+    if (dense_mode(c) && c->total_cache_size % tf)
+        return fail(PBSA_ERR_ARG, "dense mode: total_cache_size %d is not a multiple of %d tokens/frame",
+                    c->total_cache_size, tf);
     if (c->persistent_cache_size < 0) return fail(PBSA_ERR_ARG, "persistent_cache_size < 0");
     if (c->total_cache_size != c->local_cache_size + c->persistent_cache_size)
         return fail(PBSA_ERR_ARG, "total_cache_size %d != local %d + persistent %d",
@@ -80,7 +90,7 @@ int validate(const pbsa_config* c) {
     if (c->max_seq_len < tf) return fail(PBSA_ERR_ARG, "max_seq_len %d < one frame (%d)", c->max_seq_len, tf);
     const float r = c->local_block_sparse_topk_ratio;
     if (!(r > 0.f && r <= 1.f)) return fail(PBSA_ERR_ARG, "local_block_sparse_topk_ratio %g not in (0, 1]", r);
-    const int W = c->local_cache_size / tf;
+    const int W = window_tokens(c) / tf;
     const int nlmax = W * blocks_per_frame(c);
     if (nlmax > 512) return fail(PBSA_ERR_UNSUPPORTED, "%d local blocks > 512", nlmax);
     if (num_slots(c) > 1024) return fail(PBSA_ERR_UNSUPPORTED, "%d persistent slots > 1024", num_slots(c));
@@ -98,7 +108,7 @@ pbsa::Geo make_geo(const pbsa_config* c) {
     g.nby = (c->frame_h + 7) / 8;
     g.nbx = (c->frame_w + 7) / 8;
     g.nbf = g.nby * g.nbx;
-    g.W = c->local_cache_size / g.tf;
+    g.W = window_tokens(c) / g.tf;
     g.S = num_slots(c);
     return g;
 }
@@ -122,6 +132,12 @@ int check_window(const pbsa_config* c, const pbsa::Geo& g, int q_frames, int loc
 #define OPTIONAL_PTR(p)                                                       \
     do {                                                                      \
         if ((p) && !aligned16(p)) return fail(PBSA_ERR_ARG, "%s is not 16-byte aligned", #p); \
+    } while (0)
+
+// persistent-cache arguments: required when there are slots, ignored (may be NULL) when S = 0
+#define PERS_PTR(g, p)                                                        \
+    do {                                                                      \
+        if ((g).S > 0) REQUIRE_PTR(p);                                        \
     } while (0)
 
 // ------------------------------------------------------------------ tensor maps
@@ -170,6 +186,20 @@ int map_rows(CUtensorMap* m, const void* ptr, const pbsa::Geo& g, long long rows
     return PBSA_OK;
 }
 
+// The two slot-store maps (8-row and 64-row boxes).  With no slots the kernels never load
+// from them; they are then encoded over the window buffer so that every map is valid.
+int map_slots(CUtensorMap* m8, CUtensorMap* m64, const void* pers, const void* window, const pbsa::Geo& g) {
+    long long rows = (long long)g.B * g.H * g.S * 64;
+    const void* base = pers;
+    if (g.S == 0) {
+        rows = (long long)g.B * g.W * g.tf * g.H;
+        base = window;
+    }
+    int rc = map_rows(m8, base, g, rows, rows < 8 ? (int)rows : 8);
+    if (rc != PBSA_OK) return rc;
+    return map_rows(m64, base, g, rows, rows < 64 ? (int)rows : 64);
+}
+
 size_t select_ws(const pbsa::Geo& g, int q_frames) {
     return align256(sizeof(float) * (size_t)g.B * g.H * q_frames * g.nbf * g.D) +
            align256(sizeof(float) * (size_t)g.B * g.H * g.W * g.nbf * g.D);
@@ -208,7 +238,7 @@ int pbsa_blocks_per_frame(const pbsa_config* cfg) {
 
 int pbsa_window_frames(const pbsa_config* cfg) {
     if (validate(cfg) != PBSA_OK) return -1;
-    return cfg->local_cache_size / tokens_per_frame(cfg);
+    return window_tokens(cfg) / tokens_per_frame(cfg);
 }
 
 int pbsa_num_slots(const pbsa_config* cfg) {
@@ -218,7 +248,7 @@ int pbsa_num_slots(const pbsa_config* cfg) {
 
 int pbsa_topk_count(const pbsa_config* cfg, int local_frames) {
     if (validate(cfg) != PBSA_OK) return -1;
-    if (local_frames < 0 || local_frames > cfg->local_cache_size / tokens_per_frame(cfg))
+    if (local_frames < 0 || local_frames > window_tokens(cfg) / tokens_per_frame(cfg))
         return fail(PBSA_ERR_ARG, "local_frames %d out of range", local_frames);
     return topk_count(cfg, local_frames);
 }
@@ -257,6 +287,11 @@ int pbsa_select_blocks(const pbsa_config* cfg, const void* q, int q_frames, cons
     if (pbsa::score_topk_smem_bytes(g, nl) > 227 * 1024)
         return fail(PBSA_ERR_UNSUPPORTED, "%d local blocks do not fit the scoring kernel", nl);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (k == nl && !scores) {
+        cudaError_t e = pbsa::launch_select_all(g, q_frames * g.nbf, nl, idx, idx_stride, cnt, st);
+        if (e != cudaSuccess) return cuda_fail(e, "select-all kernel launch");
+        return PBSA_OK;
+    }
     float* qbar = static_cast<float*>(workspace);
     float* kbar = reinterpret_cast<float*>(static_cast<char*>(workspace) +
                                            align256(sizeof(float) * (size_t)g.B * g.H * q_frames * g.nbf * g.D));
@@ -279,9 +314,9 @@ int pbsa_attn_fwd(const pbsa_config* cfg, const void* q, int q_frames, const voi
     const pbsa::Geo g = make_geo(cfg);
     if ((rc = check_window(cfg, g, q_frames, local_frames, ring_head)) != PBSA_OK) return rc;
     REQUIRE_PTR(q);
-    REQUIRE_PTR(k_pers);
-    REQUIRE_PTR(v_pers);
-    REQUIRE_PTR(pers_len);
+    PERS_PTR(g, k_pers);
+    PERS_PTR(g, v_pers);
+    PERS_PTR(g, pers_len);
     REQUIRE_PTR(k_local);
     REQUIRE_PTR(v_local);
     REQUIRE_PTR(idx);
@@ -321,10 +356,8 @@ int pbsa_attn_fwd(const pbsa_config* cfg, const void* q, int q_frames, const voi
     if ((rc = map_tokens(&a.tm_o, out, g, (long long)g.B * q_frames)) != PBSA_OK) return rc;
     if ((rc = map_tokens(&a.tm_kl, k_local, g, (long long)g.B * g.W)) != PBSA_OK) return rc;
     if ((rc = map_tokens(&a.tm_vl, v_local, g, (long long)g.B * g.W)) != PBSA_OK) return rc;
-    if ((rc = map_rows(&a.tm_kp, k_pers, g, (long long)g.B * g.H * g.S * 64)) != PBSA_OK) return rc;
-    if ((rc = map_rows(&a.tm_vp, v_pers, g, (long long)g.B * g.H * g.S * 64)) != PBSA_OK) return rc;
-    if ((rc = map_rows(&a.tm_kp64, k_pers, g, (long long)g.B * g.H * g.S * 64, 64)) != PBSA_OK) return rc;
-    if ((rc = map_rows(&a.tm_vp64, v_pers, g, (long long)g.B * g.H * g.S * 64, 64)) != PBSA_OK) return rc;
+    if ((rc = map_slots(&a.tm_kp, &a.tm_kp64, k_pers, k_local, g)) != PBSA_OK) return rc;
+    if ((rc = map_slots(&a.tm_vp, &a.tm_vp64, v_pers, v_local, g)) != PBSA_OK) return rc;
     cudaError_t e = pbsa::launch_attn_fwd(a, with_mass, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "forward kernel launch");
     return PBSA_OK;
@@ -341,9 +374,9 @@ int pbsa_attn_bwd(const pbsa_config* cfg, const void* q, int q_frames, const voi
     const pbsa::Geo g = make_geo(cfg);
     if ((rc = check_window(cfg, g, q_frames, local_frames, ring_head)) != PBSA_OK) return rc;
     REQUIRE_PTR(q);
-    REQUIRE_PTR(k_pers);
-    REQUIRE_PTR(v_pers);
-    REQUIRE_PTR(pers_len);
+    PERS_PTR(g, k_pers);
+    PERS_PTR(g, v_pers);
+    PERS_PTR(g, pers_len);
     REQUIRE_PTR(k_local);
     REQUIRE_PTR(v_local);
     REQUIRE_PTR(idx);
@@ -352,8 +385,8 @@ int pbsa_attn_bwd(const pbsa_config* cfg, const void* q, int q_frames, const voi
     REQUIRE_PTR(lse);
     REQUIRE_PTR(dout);
     REQUIRE_PTR(dq);
-    REQUIRE_PTR(dk_pers);
-    REQUIRE_PTR(dv_pers);
+    PERS_PTR(g, dk_pers);
+    PERS_PTR(g, dv_pers);
     REQUIRE_PTR(dk_local);
     REQUIRE_PTR(dv_local);
     REQUIRE_PTR(workspace);
@@ -387,10 +420,8 @@ int pbsa_attn_bwd(const pbsa_config* cfg, const void* q, int q_frames, const voi
     if ((rc = map_tokens(&a.tm_do, dout, g, (long long)g.B * q_frames)) != PBSA_OK) return rc;
     if ((rc = map_tokens(&a.tm_kl, k_local, g, (long long)g.B * g.W)) != PBSA_OK) return rc;
     if ((rc = map_tokens(&a.tm_vl, v_local, g, (long long)g.B * g.W)) != PBSA_OK) return rc;
-    if ((rc = map_rows(&a.tm_kp, k_pers, g, (long long)g.B * g.H * g.S * 64)) != PBSA_OK) return rc;
-    if ((rc = map_rows(&a.tm_vp, v_pers, g, (long long)g.B * g.H * g.S * 64)) != PBSA_OK) return rc;
-    if ((rc = map_rows(&a.tm_kp64, k_pers, g, (long long)g.B * g.H * g.S * 64, 64)) != PBSA_OK) return rc;
-    if ((rc = map_rows(&a.tm_vp64, v_pers, g, (long long)g.B * g.H * g.S * 64, 64)) != PBSA_OK) return rc;
+    if ((rc = map_slots(&a.tm_kp, &a.tm_kp64, k_pers, k_local, g)) != PBSA_OK) return rc;
+    if ((rc = map_slots(&a.tm_vp, &a.tm_vp64, v_pers, v_local, g)) != PBSA_OK) return rc;
     cudaError_t e = pbsa::launch_attn_bwd(a, static_cast<cudaStream_t>(stream));
     if (e == cudaErrorNotSupported) return fail(PBSA_ERR_UNSUPPORTED, "backward kernel not built");
     if (e != cudaSuccess) return cuda_fail(e, "backward kernel launch");
@@ -413,11 +444,11 @@ int pbsa_cache_update(const pbsa_config* cfg, const void* k_local, const void* v
     REQUIRE_PTR(k_local);
     REQUIRE_PTR(v_local);
     REQUIRE_PTR(mass_local);
-    REQUIRE_PTR(k_pers);
-    REQUIRE_PTR(v_pers);
-    REQUIRE_PTR(pers_len);
-    REQUIRE_PTR(pers_score);
-    REQUIRE_PTR(pers_src);
+    PERS_PTR(g, k_pers);
+    PERS_PTR(g, v_pers);
+    PERS_PTR(g, pers_len);
+    PERS_PTR(g, pers_score);
+    PERS_PTR(g, pers_src);
     REQUIRE_PTR(upd);
     REQUIRE_PTR(n_upd);
     cudaError_t e = pbsa::launch_cache_update(

@@ -70,6 +70,8 @@ cudaError_t launch_score_topk(const Geo& g, const float* qbar, const float* kbar
                               int nl, int k, int32_t* idx, int idx_stride, int32_t* cnt,
                               float* scores, cudaStream_t st);
 size_t score_topk_smem_bytes(const Geo& g, int nl);
+cudaError_t launch_select_all(const Geo& g, int qb, int nl, int32_t* idx, int idx_stride, int32_t* cnt,
+                              cudaStream_t st);
 
 cudaError_t launch_attn_fwd(const FwdArgs& a, bool with_mass, cudaStream_t st);
 size_t attn_fwd_smem_bytes(const Geo& g, int ucap);

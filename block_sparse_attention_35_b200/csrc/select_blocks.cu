@@ -192,7 +192,24 @@ __global__ void __launch_bounds__(256) score_topk_kernel(ScoreParams p) {
     }
 }
 
+// Every window block selected (k = N_L, no scores asked for): the list is 0..N_L-1.
+__global__ void __launch_bounds__(256) select_all_kernel(int32_t* __restrict__ idx, int idx_stride,
+                                                         int32_t* __restrict__ cnt, long long rows, int nl) {
+    const long long r = (long long)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
+    if (r >= rows) return;
+    const int lane = threadIdx.x & 31;
+    for (int j = lane; j < nl; j += 32) idx[r * idx_stride + j] = j;
+    if (lane == 0) cnt[r] = nl;
+}
+
 }  // namespace
+
+cudaError_t launch_select_all(const Geo& g, int qb, int nl, int32_t* idx, int idx_stride, int32_t* cnt,
+                              cudaStream_t st) {
+    const long long rows = (long long)g.B * g.H * qb;   // one warp per (b, h, query block)
+    select_all_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(idx, idx_stride, cnt, rows, nl);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_pool(const Geo& g, const __nv_bfloat16* q, int q_frames,
                         const __nv_bfloat16* k_local, int local_frames, int ring_head,

@@ -56,6 +56,13 @@ extern "C" PBSA_API int pbsa_select_blocks_noalloc(const pbsa_config* cfg, const
     int rc = pbsa::api_prepare_select(cfg, q, q_frames, k_local, local_frames, ring_head, idx, idx_stride,
                                       cnt, scores, &g, &k, &need, &key_off);
     if (rc != PBSA_OK) return rc;
+    // every window block selected and no scores asked for: no scratch needed
+    if (k == local_frames * g.nbf && !scores) {
+        cudaError_t e = pbsa::launch_select_all(g, q_frames * g.nbf, k, idx, idx_stride, cnt,
+                                                static_cast<cudaStream_t>(stream));
+        if (e != cudaSuccess) return pbsa::api_cuda_fail(e, "select-all kernel launch");
+        return PBSA_OK;
+    }
     if (need > kScratchBytes)
         return pbsa::api_fail(PBSA_ERR_UNSUPPORTED,
                               "selection needs more scratch than the 8 MiB static buffer of "

@@ -26,6 +26,7 @@ PBSA_ERR_TIMEOUT = -4
 PBSA_ERR_DEVICE_CHECK = -5
 PBSA_ERR_WORKSPACE = -6
 PBSA_OP_SELECT, PBSA_OP_FWD, PBSA_OP_BWD, PBSA_OP_UPDATE = 0, 1, 2, 3
+PBSA_KV_CACHE_SPARSE_FORCING, PBSA_KV_CACHE_DENSE = 0, 1
 
 
 class PBSAError(RuntimeError):
@@ -52,7 +53,7 @@ def make_config(B, H, D, frame_h, frame_w, total_cache_size, local_cache_size,
                 use_local_block_sparse_attn=True, sparse_kv_block_size=(1, 8, 8),
                 kv_cache_mode="sparse_forcing") -> pbsa_config:
     """Builds a pbsa_config from the SparseForcingAttention constructor arguments."""
-    modes = {"sparse_forcing": 0}
+    modes = {"sparse_forcing": PBSA_KV_CACHE_SPARSE_FORCING, "dense": PBSA_KV_CACHE_DENSE}
     if kv_cache_mode not in modes:
         raise PBSAError(PBSA_ERR_UNSUPPORTED, f"kv_cache_mode {kv_cache_mode!r}")
     bt, bh, bw = sparse_kv_block_size

@@ -69,6 +69,11 @@ extern "C" {
 #define PBSA_ERR_WORKSPACE (-6)    /* workspace too small */
 
 #define PBSA_KV_CACHE_SPARSE_FORCING 0 /* kv_cache_mode="sparse_forcing" */
+/* kv_cache_mode="dense" (a reading: the project page names only "sparse_forcing"; this is
+ * the plain cache the pages compare against): the window is the whole total_cache_size,
+ * there are no persistent slots (S = 0), every window block is attended, and a slide
+ * simply drops the oldest frames.  Persistent pointers may then be NULL. */
+#define PBSA_KV_CACHE_DENSE 1
 
 /* Operation ids for pbsa_workspace_size. */
 #define PBSA_OP_SELECT 0
@@ -89,7 +94,7 @@ typedef struct pbsa_config {
     int local_cache_size;        /* tokens; a whole number of frames */
     int persistent_cache_size;   /* tokens */
     int max_seq_len;             /* tokens; bounds q_frames * T_f */
-    int kv_cache_mode;           /* PBSA_KV_CACHE_SPARSE_FORCING */
+    int kv_cache_mode;           /* PBSA_KV_CACHE_SPARSE_FORCING or PBSA_KV_CACHE_DENSE */
     int use_local_block_sparse_attn; /* 0: every local block is attended */
     float local_block_sparse_topk_ratio; /* in (0, 1] */
 } pbsa_config;
@@ -100,14 +105,16 @@ typedef struct pbsa_config {
 PBSA_API int pbsa_validate_config(const pbsa_config* cfg);
 /* NB_f, blocks per frame. */
 PBSA_API int pbsa_blocks_per_frame(const pbsa_config* cfg);
-/* W, frame slots of the local ring (local_cache_size / T_f). */
+/* W, frame slots of the local ring (local_cache_size / T_f; total_cache_size / T_f in
+ * dense mode). */
 PBSA_API int pbsa_window_frames(const pbsa_config* cfg);
 /* S, persistent slots: persistent_cache_size / T_f * NB_f when that divides, else
- * ceil(persistent_cache_size / 64). */
+ * ceil(persistent_cache_size / 64); 0 in dense mode. */
 PBSA_API int pbsa_num_slots(const pbsa_config* cfg);
 /* k, local blocks attended per query block for a window of local_frames frames:
- * N_L = local_frames * NB_f; k = N_L when use_local_block_sparse_attn is 0, else
- * clamp(ceil(ratio * N_L), 1, N_L). */
+ * N_L = local_frames * NB_f; k = N_L when use_local_block_sparse_attn is 0 or in dense
+ * mode, else clamp(ceil(ratio * N_L), 1, N_L).  When k = N_L and no scores are asked for,
+ * pbsa_select_blocks writes the full ascending list without scoring. */
 PBSA_API int pbsa_topk_count(const pbsa_config* cfg, int local_frames);
 /* Workspace bytes needed by operation `op` (PBSA_OP_*) for a chunk of q_frames frames. */
 PBSA_API size_t pbsa_workspace_size(const pbsa_config* cfg, int op, int q_frames);

@@ -78,6 +78,23 @@ def n_slots(persistent_cache_size: int, frame_h: int, frame_w: int, bh=8, bw=8) 
     return -(-persistent_cache_size // (bh * bw))
 
 
+def cache_geometry(kv_cache_mode: str, total_cache_size: int, local_cache_size: int,
+                   persistent_cache_size: int, frame_h: int, frame_w: int, bh=8, bw=8):
+    """(window frames W, persistent slots S, every window block attended?) of a cache mode.
+
+    kv_cache_mode="sparse_forcing" (project page, constructor default): a window of
+    local_cache_size tokens plus the persistent slots.  "dense" (reading: the plain cache
+    the pages compare Sparse Forcing with; the page names no other mode): one window of
+    total_cache_size tokens, no persistent slots, every block attended, eviction drops.
+    """
+    tf = frame_h * frame_w
+    if kv_cache_mode == "dense":
+        return total_cache_size // tf, 0, True
+    if kv_cache_mode != "sparse_forcing":
+        raise ValueError(kv_cache_mode)
+    return local_cache_size // tf, n_slots(persistent_cache_size, frame_h, frame_w, bh, bw), False
+
+
 # ---------------------------------------------------------------------------------------
 # Block selection (project page: learned top-k selection, local_block_sparse_topk_ratio;
 # pith abstract: "dynamically selected local neighborhood")

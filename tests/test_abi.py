@@ -102,3 +102,20 @@ def test_argument_errors_are_reported_before_any_launch():
     rc = lib.pbsa_cache_update(ctypes.byref(cfg), 256, 256, 3, 0, 256, 4, 0, 256, 256, 256,
                                256, 256, 256, 256, None, 0, None)
     assert rc == P.PBSA_ERR_ARG and "n_evict_frames" in P.pbsa_last_error()
+
+
+def test_dense_cache_mode_queries():
+    wl = WORKLOADS["decode"]
+    cfg = config(wl, kv_cache_mode="dense")
+    P.pbsa_validate_config(cfg)
+    W, S, _ = orc.cache_geometry("dense", wl.total_cache_size, wl.local_cache_size,
+                                 wl.persistent_cache_size, wl.frame_h, wl.frame_w)
+    assert P.pbsa_window_frames(cfg) == W == 12
+    assert P.pbsa_num_slots(cfg) == S == 0
+    assert P.pbsa_topk_count(cfg, 12) == 12 * 28          # every block of the window
+    assert P.pbsa_workspace_size(cfg, P.PBSA_OP_FWD, 3) > 0
+    bad = config(wl, kv_cache_mode="dense")
+    bad.total_cache_size, bad.persistent_cache_size = 18720 + 100, 9360 + 100
+    with pytest.raises(P.PBSAError) as e:
+        P.pbsa_validate_config(bad)
+    assert e.value.code == P.PBSA_ERR_ARG

@@ -444,3 +444,35 @@ def test_merge_hand_example_empty_slots_fill_before_dropped_ones():
     assert list(r["pers_len"][0, 0]) == [64, 64, 64, 32]
     assert list(r["pers_score"][0, 0]) == [4.0, 1.0, 5.0, 3.0]
     assert list(r["pers_src"][0, 0]) == [14, 1001, 1002, 15]
+
+
+def test_dense_cache_mode_geometry():
+    # page sizes: the dense window is the whole 18720-token cache (12 frames of 1560)
+    assert orc.cache_geometry("dense", 18720, 9360, 9360, 30, 52) == (12, 0, True)
+    assert orc.cache_geometry("sparse_forcing", 18720, 9360, 9360, 30, 52) == (6, 168, False)
+    with pytest.raises(ValueError):
+        orc.cache_geometry("paged", 18720, 9360, 9360, 30, 52)
+
+
+def test_dense_cache_mode_forward_is_dense_attention_over_the_window():
+    # dense mode = every window block selected and no persistent slots: plain attention
+    t = _tiny(filled=())
+    W, S, select_all = orc.cache_geometry("dense", t["kw"].shape[1], t["kw"].shape[1], 0,
+                                          t["fh"], t["fw"])
+    assert S == 0 and select_all
+    idx, _ = orc.select_blocks(t["q"], t["kw"], t["fh"], t["fw"], ratio=0.25,
+                               use_sparse=not select_all)
+    nl = idx.shape[-1]
+    assert (idx == np.arange(nl)).all()
+    B, nq, H, D = t["q"].shape
+    kp0 = np.zeros((B, H, 0, 64, D))
+    O, lse, mp, ml = orc.attn_fwd(t["q"], kp0, kp0, np.zeros((B, H, 0), np.int64), t["kw"],
+                                  t["vw"], idx, t["fh"], t["fw"])
+    for b in range(B):
+        for h in range(H):
+            qt = torch.tensor(t["q"][b, :, h])[None, None]
+            kt = torch.tensor(t["kw"][b, :, h])[None, None]
+            vt = torch.tensor(t["vw"][b, :, h])[None, None]
+            want = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt)[0, 0].numpy()
+            assert np.allclose(O[b, :, h], want, rtol=0, atol=1e-12)
+    assert mp.size == 0
