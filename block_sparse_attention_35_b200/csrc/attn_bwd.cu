@@ -291,11 +291,31 @@ __global__ void __launch_bounds__(kThreads, 1) dkdv_kernel(const __grid_constant
         int issued = 0;
         for (int j = 0; j < n_items; ++j) {
             const int st = j % kNst;
+            const int qt = qtl[j];
+            // lse (log2 units) and Delta of the tile's 128 query rows, read from global memory
+            // before waiting for the stage so that their latency overlaps the wait; +inf lse
+            // masks padding rows
+            float l2v[4], dlv[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int r = lane + 32 * u;
+                const int hq = r >> 6, qb = 2 * qt + hq, rr = r & 63;
+                l2v[u] = CUDART_INF_F;
+                dlv[u] = 0.f;
+                if (qb < qb_total) {
+                    const int f = qb / g.nbf, i = qb % g.nbf;
+                    const int y = 8 * (i / g.nbx) + (rr >> 3), x = 8 * (i % g.nbx) + (rr & 7);
+                    if (y < g.fh && x < g.fw) {
+                        const size_t t = (size_t)bh * nq + f * g.tf + y * g.fw + x;
+                        l2v[u] = a.lse[t] * kLog2e;
+                        dlv[u] = a.delta[t];
+                    }
+                }
+            }
             if (j >= kNst) {
                 const bool w = __all_sync(0xffffffffu, mbar_wait(&qd_empty[st], ((j / kNst) - 1) & 1, abort_flag, a.status));
                 if (!w) break;
             }
-            const int qt = qtl[j];
             if (lane == 0) {
                 mbar_arrive_expect_tx(&qd_full[st], 2 * TILE);
                 for (int hq = 0; hq < 2; ++hq) {
@@ -309,21 +329,10 @@ __global__ void __launch_bounds__(kThreads, 1) dkdv_kernel(const __grid_constant
                     }
                 }
             }
-            // lse (log2 units) and Delta of the tile's 128 query rows; +inf lse masks padding
-            for (int r = lane; r < 128; r += 32) {
-                const int hq = r >> 6, qb = 2 * qt + hq, rr = r & 63;
-                float l2 = CUDART_INF_F, dl = 0.f;
-                if (qb < qb_total) {
-                    const int f = qb / g.nbf, i = qb % g.nbf;
-                    const int y = 8 * (i / g.nbx) + (rr >> 3), x = 8 * (i % g.nbx) + (rr & 7);
-                    if (y < g.fh && x < g.fw) {
-                        const size_t t = (size_t)bh * nq + f * g.tf + y * g.fw + x;
-                        l2 = a.lse[t] * kLog2e;
-                        dl = a.delta[t];
-                    }
-                }
-                s_lse[st * 128 + r] = l2;
-                s_dl[st * 128 + r] = dl;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                s_lse[st * 128 + lane + 32 * u] = l2v[u];
+                s_dl[st * 128 + lane + 32 * u] = dlv[u];
             }
             mbar_arrive(&qd_full[st]);
             ++issued;
@@ -414,8 +423,8 @@ __global__ void __launch_bounds__(kThreads, 1) dkdv_kernel(const __grid_constant
             if (!wwait(sdp_full, j & 1)) { ok = false; break; }
             tc_fence_after();
             const bool sel = key_valid && ((qsel[j] >> (2 * kbr + hq)) & 1);
-            const float4* lse4 = reinterpret_cast<const float4*>(s_lse + st * 128 + c0);
-            const float4* dl4 = reinterpret_cast<const float4*>(s_dl + st * 128 + c0);
+            const float l_mine = s_lse[st * 128 + c0 + lane];
+            const float d_mine = s_dl[st * 128 + c0 + lane];
             uint32_t pk[kCw / 2], dk[kCw / 2];
 #pragma unroll
             for (int sc = 0; sc < kCw / 16; ++sc) {
@@ -425,10 +434,12 @@ __global__ void __launch_bounds__(kThreads, 1) dkdv_kernel(const __grid_constant
                 tmem_ld_wait();
 #pragma unroll
                 for (int e4 = 0; e4 < 4; ++e4) {
-                    const float4 l4 = lse4[4 * sc + e4];
-                    const float4 d4 = dl4[4 * sc + e4];
-                    const float ls[4] = {l4.x, l4.y, l4.z, l4.w};
-                    const float ds[4] = {d4.x, d4.y, d4.z, d4.w};
+                    float ls[4], ds[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        ls[u] = __shfl_sync(0xffffffffu, l_mine, 16 * sc + 4 * e4 + u);
+                        ds[u] = __shfl_sync(0xffffffffu, d_mine, 16 * sc + 4 * e4 + u);
+                    }
                     float p[4], d[4];
 #pragma unroll
                     for (int u = 0; u < 4; ++u) {
