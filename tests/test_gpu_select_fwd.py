@@ -149,3 +149,25 @@ def test_decode_full_size_sampled(cuda_dev):
 def test_decode_full_size_one_head_mass(cuda_dev):
     wl = dataclasses.replace(WORKLOADS["decode"], H=1)
     _run_case(wl, cuda_dev)
+
+
+# Long-horizon sweep shapes (H12 D128, 30x52 frames): persistent 4680 / 9360 / 18720 tokens
+# (84 / 168 / 336 slots), window 4680 / 9360 tokens (3 / 6 frames), ratio 1/16 .. 1/4,
+# batch 1 and 4; the extremes of the grid, in the launch configuration of the benchmark,
+# with sampled query blocks of sampled (batch, head) pairs recomputed by the oracle.
+SWEEP = [
+    dict(persistent_cache_size=4680, local_cache_size=4680, topk_ratio=1 / 16, B=1),
+    dict(persistent_cache_size=18720, local_cache_size=9360, topk_ratio=1 / 4, B=1),
+    dict(persistent_cache_size=9360, local_cache_size=4680, topk_ratio=1 / 8, B=4),
+    dict(persistent_cache_size=18720, local_cache_size=4680, topk_ratio=1 / 16, B=4),
+]
+
+
+@pytest.mark.parametrize("case", range(len(SWEEP)))
+def test_long_horizon_sweep_shapes_sampled(cuda_dev, case):
+    over = SWEEP[case]
+    wl = dataclasses.replace(WORKLOADS["decode"], name=f"sweep{case}", seed=20 + case,
+                             total_cache_size=over["persistent_cache_size"] + over["local_cache_size"],
+                             **over)
+    heads = [(0, 0), (wl.B - 1, 5), (wl.B // 2, 11)]
+    _run_case(wl, cuda_dev, qblocks=[0, 13, 27, 50, 83], heads=heads)
