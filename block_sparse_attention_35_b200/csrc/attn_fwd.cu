@@ -11,7 +11,8 @@
 // ("sides" A and B, two blocks each, every block a 64-row 5-D TMA box; ragged edge blocks
 // are zero-filled on load and clipped on store).  Key tiles are 128 keys:
 //   * persistent tiles (shared by both sides): the occupied slots' valid rows compacted
-//     into a stream of 8-row groups (slot lengths are multiples of 8), 16 groups per tile;
+//     into a stream of 8-row groups (slot lengths are multiples of 8), 16 groups per tile,
+//     loaded as one 64-row TMA box wherever eight groups are contiguous rows (a full slot);
 //   * local tiles (one side each): the union of that side's two selections, two 8x8 key
 //     blocks per tile; columns the row's query block did not select, or outside the frame,
 //     are masked.  A-tiles and B-tiles alternate in the stream.
@@ -23,7 +24,11 @@
 // Warp roles (384 threads): warps 0-3 softmax of side A, 4-7 side B (one query row per
 // thread), warp 8 K (and Q) producer, warp 9 V producer, warp 10 MMA issuer, warp 11 idle.  K and V
 // stages have separate full/empty barriers.  O is rescaled only when a row maximum grows by
-// more than 2^8.  Mass: each row emits, per slot/block it saw, log2 of its partial
+// more than 2^8; so the softmax first exponentiates half of the row against the running
+// reference while taking the tile's row maximum in the same pass, and only a warp with a
+// row that needs a new reference rescales O and redoes that half from S (still intact in
+// TMEM).  Each half's P is stored as soon as it is packed.  Mass: each row emits, per
+// slot/block it saw, log2 of its partial
 // probability sum (relative to its running maximum) into workspace; once the final
 // log-sum-exp is known the side converts them, sums over its rows and adds one value per
 // slot/block to the global mass arrays.

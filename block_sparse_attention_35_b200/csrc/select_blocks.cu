@@ -131,13 +131,22 @@ __global__ void __launch_bounds__(256) score_topk_kernel(ScoreParams p) {
     const int bh = b * g.H + h;
     const int nl = p.nl;
     float* kb = sm;                               // [nl][D+1]
-    float* qs = kb + (size_t)nl * (D + 1);        // [8][D]
+    float* qs = kb + (((size_t)nl * (D + 1) + 3) & ~(size_t)3);  // [8][D], 16-byte aligned
     float* sc = qs + kQbPerCta * D;               // [8][nl]
 
-    const float* ksrc = p.kbar + (size_t)bh * nl * D;
-    for (int e = threadIdx.x; e < nl * D; e += blockDim.x) {
-        const int j = e / D, d = e % D;
-        kb[j * (D + 1) + d] = ksrc[e];
+    // 16-byte loads, several in flight per thread (the copy is latency-bound otherwise);
+    // rows are stored padded to D + 1 floats so that the dot products below are conflict-free
+    const float4* ksrc = reinterpret_cast<const float4*>(p.kbar + (size_t)bh * nl * D);
+    const int n4 = nl * D / 4;
+#pragma unroll 4
+    for (int e = threadIdx.x; e < n4; e += blockDim.x) {
+        const float4 v = __ldg(ksrc + e);
+        const int j = (4 * e) / D, d = (4 * e) % D;
+        float* dst = kb + j * (D + 1) + d;
+        dst[0] = v.x;
+        dst[1] = v.y;
+        dst[2] = v.z;
+        dst[3] = v.w;
     }
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int qb = blockIdx.x * kQbPerCta + warp;
@@ -153,9 +162,16 @@ __global__ void __launch_bounds__(256) score_topk_kernel(ScoreParams p) {
     const float inv_sqrt_d = 1.0f / sqrtf(static_cast<float>(D));
     for (int j = lane; j < nl; j += 32) {
         const float* kr = kb + j * (D + 1);
-        float acc = 0.f;
-        for (int d = 0; d < D; ++d) acc = fmaf(qrow[d], kr[d], acc);
-        srow[j] = acc * inv_sqrt_d;
+        float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll 8
+        for (int d = 0; d < D; d += 4) {
+            const float4 q4 = *reinterpret_cast<const float4*>(qrow + d);
+            acc0 = fmaf(q4.x, kr[d], acc0);
+            acc1 = fmaf(q4.y, kr[d + 1], acc1);
+            acc0 = fmaf(q4.z, kr[d + 2], acc0);
+            acc1 = fmaf(q4.w, kr[d + 3], acc1);
+        }
+        srow[j] = (acc0 + acc1) * inv_sqrt_d;
     }
     __syncwarp();
 
@@ -222,7 +238,8 @@ cudaError_t launch_pool(const Geo& g, const __nv_bfloat16* q, int q_frames,
 }
 
 size_t score_topk_smem_bytes(const Geo& g, int nl) {
-    return sizeof(float) * ((size_t)nl * (g.D + 1) + (size_t)kQbPerCta * g.D + (size_t)kQbPerCta * nl);
+    return sizeof(float) * ((((size_t)nl * (g.D + 1) + 3) & ~(size_t)3) + (size_t)kQbPerCta * g.D +
+                            (size_t)kQbPerCta * nl);
 }
 
 cudaError_t launch_score_topk(const Geo& g, const float* qbar, const float* kbar, int qb, int nl,
