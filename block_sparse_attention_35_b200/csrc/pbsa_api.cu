@@ -296,10 +296,60 @@ int pbsa_select_blocks(const pbsa_config* cfg, const void* q, int q_frames, cons
     float* kbar = reinterpret_cast<float*>(static_cast<char*>(workspace) +
                                            align256(sizeof(float) * (size_t)g.B * g.H * q_frames * g.nbf * g.D));
     cudaError_t e = pbsa::launch_pool(g, static_cast<const __nv_bfloat16*>(q), q_frames,
-                                      static_cast<const __nv_bfloat16*>(k_local), local_frames, ring_head,
+                                      static_cast<const __nv_bfloat16*>(k_local), ring_head, local_frames,
                                       qbar, kbar, st);
     if (e != cudaSuccess) return cuda_fail(e, "pool kernel launch");
-    e = pbsa::launch_score_topk(g, qbar, kbar, q_frames * g.nbf, nl, k, idx, idx_stride, cnt, scores, st);
+    e = pbsa::launch_score_topk(g, qbar, kbar, ring_head, q_frames * g.nbf, nl, k, idx, idx_stride, cnt, scores, st);
+    if (e != cudaSuccess) return cuda_fail(e, "score/top-k kernel launch");
+    return PBSA_OK;
+}
+
+int pbsa_pool_keys(const pbsa_config* cfg, const void* k_local, int first_slot, int n_frames, float* kbar,
+                   void* stream) {
+    int rc = validate(cfg);
+    if (rc != PBSA_OK) return rc;
+    const pbsa::Geo g = make_geo(cfg);
+    if (first_slot < 0 || first_slot >= g.W) return fail(PBSA_ERR_ARG, "first_slot %d not in [0, %d)", first_slot, g.W);
+    if (n_frames < 0 || n_frames > g.W) return fail(PBSA_ERR_ARG, "n_frames %d not in [0, %d]", n_frames, g.W);
+    REQUIRE_PTR(k_local);
+    REQUIRE_PTR(kbar);
+    cudaError_t e = pbsa::launch_pool(g, nullptr, 0, static_cast<const __nv_bfloat16*>(k_local), first_slot,
+                                      n_frames, nullptr, kbar, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "pool kernel launch");
+    return PBSA_OK;
+}
+
+int pbsa_select_blocks_pooled(const pbsa_config* cfg, const void* q, int q_frames, const float* kbar,
+                              int local_frames, int ring_head, int32_t* idx, int idx_stride, int32_t* cnt,
+                              float* scores, void* workspace, size_t workspace_bytes, void* stream) {
+    int rc = validate(cfg);
+    if (rc != PBSA_OK) return rc;
+    const pbsa::Geo g = make_geo(cfg);
+    if ((rc = check_window(cfg, g, q_frames, local_frames, ring_head)) != PBSA_OK) return rc;
+    REQUIRE_PTR(q);
+    REQUIRE_PTR(kbar);
+    REQUIRE_PTR(idx);
+    REQUIRE_PTR(cnt);
+    OPTIONAL_PTR(scores);
+    const int k = topk_count(cfg, local_frames);
+    if (idx_stride < k) return fail(PBSA_ERR_ARG, "idx_stride %d < k %d", idx_stride, k);
+    const int nl = local_frames * g.nbf;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (k == nl && !scores) {
+        cudaError_t e = pbsa::launch_select_all(g, q_frames * g.nbf, nl, idx, idx_stride, cnt, st);
+        if (e != cudaSuccess) return cuda_fail(e, "select-all kernel launch");
+        return PBSA_OK;
+    }
+    REQUIRE_PTR(workspace);
+    const size_t need = align256(sizeof(float) * (size_t)g.B * g.H * q_frames * g.nbf * g.D);
+    if (workspace_bytes < need) return fail(PBSA_ERR_WORKSPACE, "workspace %zu < %zu bytes", workspace_bytes, need);
+    if (pbsa::score_topk_smem_bytes(g, nl) > 227 * 1024)
+        return fail(PBSA_ERR_UNSUPPORTED, "%d local blocks do not fit the scoring kernel", nl);
+    float* qbar = static_cast<float*>(workspace);
+    cudaError_t e = pbsa::launch_pool(g, static_cast<const __nv_bfloat16*>(q), q_frames, nullptr, 0, 0, qbar,
+                                      nullptr, st);
+    if (e != cudaSuccess) return cuda_fail(e, "pool kernel launch");
+    e = pbsa::launch_score_topk(g, qbar, kbar, ring_head, q_frames * g.nbf, nl, k, idx, idx_stride, cnt, scores, st);
     if (e != cudaSuccess) return cuda_fail(e, "score/top-k kernel launch");
     return PBSA_OK;
 }

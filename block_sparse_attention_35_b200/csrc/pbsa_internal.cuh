@@ -63,11 +63,13 @@ struct BwdArgs {
 };
 
 // Launchers (return a cudaError_t from the launch).
+// Pools q_frames query frames (may be 0) and the K frames in ring slots k_first.. (k_frames of
+// them, mod W; may be 0); key means go to kbar by physical ring slot [B, H, W*NB_f, D].
 cudaError_t launch_pool(const Geo& g, const __nv_bfloat16* q, int q_frames,
-                        const __nv_bfloat16* k_local, int local_frames, int ring_head,
+                        const __nv_bfloat16* k_local, int k_first, int k_frames,
                         float* qbar, float* kbar, cudaStream_t st);
-cudaError_t launch_score_topk(const Geo& g, const float* qbar, const float* kbar, int qb,
-                              int nl, int k, int32_t* idx, int idx_stride, int32_t* cnt,
+cudaError_t launch_score_topk(const Geo& g, const float* qbar, const float* kbar, int ring_head,
+                              int qb, int nl, int k, int32_t* idx, int idx_stride, int32_t* cnt,
                               float* scores, cudaStream_t st);
 size_t score_topk_smem_bytes(const Geo& g, int nl);
 cudaError_t launch_select_all(const Geo& g, int qb, int nl, int32_t* idx, int idx_stride, int32_t* cnt,

@@ -10,7 +10,9 @@
 //  1. pool_kernel: one CTA per (block, batch); each thread owns 8 consecutive channels of
 //     the token's [H, D] row and streams the block's valid tokens with 16-byte loads, so a
 //     CTA reads whole 3 KB token rows (all heads) - fully coalesced, one HBM pass over Q
-//     and the window's K.  Means go to fp32 workspace.
+//     and the window's K.  Means go to fp32 workspace; key means are stored by physical
+//     ring slot, so a caller can keep them across chunks and pool only the frames it
+//     appends (pbsa_pool_keys + pbsa_select_blocks_pooled).
 //  2. score_topk_kernel: one CTA per (8 query blocks, head, batch); the head's pooled keys
 //     sit in shared memory (rows padded to D+1 floats: conflict-free), one warp per query
 //     block computes its N_L scores, ranks every candidate by counting the candidates that
@@ -29,15 +31,15 @@ struct PoolParams {
     Geo g;
     const __nv_bfloat16* q;
     const __nv_bfloat16* kl;
-    int q_frames, local_frames, ring_head;
+    int q_frames;           // query frames to pool (0: none)
+    int k_first, k_frames;  // ring slots k_first, k_first+1, ... (mod W) of K to pool
     float* qbar;  // [B, H, QB, D]
-    float* kbar;  // [B, H, NL, D]
+    float* kbar;  // [B, H, W*NB_f, D], by physical ring slot
 };
 
 __global__ void __launch_bounds__(1024) pool_kernel(PoolParams p) {
     const Geo& g = p.g;
     const int qb_total = p.q_frames * g.nbf;
-    const int nl = p.local_frames * g.nbf;
     const int blk = blockIdx.x;
     const int b = blockIdx.y;
     const int hd = g.H * g.D;
@@ -57,15 +59,14 @@ __global__ void __launch_bounds__(1024) pool_kernel(PoolParams p) {
         local_id = blk;
         n_of_kind = qb_total;
     } else {
-        const int j = blk - qb_total;  // logical window block id
-        const int pos = j / g.nbf;
-        const int phys = (p.ring_head + pos) % g.W;
+        const int j = blk - qb_total;  // j-th block of the K frames being pooled
+        const int phys = (p.k_first + j / g.nbf) % g.W;
         frame = (long long)b * g.W + phys;
         i_in_frame = j % g.nbf;
         src = p.kl;
         dst = p.kbar;
-        local_id = j;
-        n_of_kind = nl;
+        local_id = phys * g.nbf + i_in_frame;
+        n_of_kind = g.W * g.nbf;
     }
     const int by = i_in_frame / g.nbx, bx = i_in_frame % g.nbx;
     const int y0 = by * 8, x0 = bx * 8;
@@ -115,7 +116,8 @@ constexpr int kMaxChunks = 16; // candidates per warp lane: N_L <= 512
 struct ScoreParams {
     Geo g;
     const float* qbar;
-    const float* kbar;
+    const float* kbar;  // [B, H, W*NB_f, D] by physical ring slot
+    int ring_head;
     int qb_total, nl, k;
     int32_t* idx;
     int idx_stride;
@@ -136,12 +138,14 @@ __global__ void __launch_bounds__(256) score_topk_kernel(ScoreParams p) {
 
     // 16-byte loads, several in flight per thread (the copy is latency-bound otherwise);
     // rows are stored padded to D + 1 floats so that the dot products below are conflict-free
-    const float4* ksrc = reinterpret_cast<const float4*>(p.kbar + (size_t)bh * nl * D);
+    // logical window block j (oldest frame first) is ring row ((ring_head + j / NB_f) % W, j % NB_f)
+    const float* kbh = p.kbar + (size_t)bh * g.W * g.nbf * D;
     const int n4 = nl * D / 4;
 #pragma unroll 4
     for (int e = threadIdx.x; e < n4; e += blockDim.x) {
-        const float4 v = __ldg(ksrc + e);
         const int j = (4 * e) / D, d = (4 * e) % D;
+        const int row = ((p.ring_head + j / g.nbf) % g.W) * g.nbf + j % g.nbf;
+        const float4 v = __ldg(reinterpret_cast<const float4*>(kbh + (size_t)row * D + d));
         float* dst = kb + j * (D + 1) + d;
         dst[0] = v.x;
         dst[1] = v.y;
@@ -228,10 +232,11 @@ cudaError_t launch_select_all(const Geo& g, int qb, int nl, int32_t* idx, int id
 }
 
 cudaError_t launch_pool(const Geo& g, const __nv_bfloat16* q, int q_frames,
-                        const __nv_bfloat16* k_local, int local_frames, int ring_head,
+                        const __nv_bfloat16* k_local, int k_first, int k_frames,
                         float* qbar, float* kbar, cudaStream_t st) {
-    PoolParams p{g, q, k_local, q_frames, local_frames, ring_head, qbar, kbar};
-    const int nblk = (q_frames + local_frames) * g.nbf;
+    PoolParams p{g, q, k_local, q_frames, k_first, k_frames, qbar, kbar};
+    const int nblk = (q_frames + k_frames) * g.nbf;
+    if (nblk == 0) return cudaSuccess;
     const int threads = (g.H * g.D / 8 + 31) / 32 * 32;
     pool_kernel<<<dim3(nblk, g.B), threads, 0, st>>>(p);
     return cudaGetLastError();
@@ -242,10 +247,10 @@ size_t score_topk_smem_bytes(const Geo& g, int nl) {
                             (size_t)kQbPerCta * nl);
 }
 
-cudaError_t launch_score_topk(const Geo& g, const float* qbar, const float* kbar, int qb, int nl,
-                              int k, int32_t* idx, int idx_stride, int32_t* cnt, float* scores,
+cudaError_t launch_score_topk(const Geo& g, const float* qbar, const float* kbar, int ring_head, int qb,
+                              int nl, int k, int32_t* idx, int idx_stride, int32_t* cnt, float* scores,
                               cudaStream_t st) {
-    ScoreParams p{g, qbar, kbar, qb, nl, k, idx, idx_stride, cnt, scores};
+    ScoreParams p{g, qbar, kbar, ring_head, qb, nl, k, idx, idx_stride, cnt, scores};
     const size_t smem = score_topk_smem_bytes(g, nl);
     cudaError_t e = cudaFuncSetAttribute(score_topk_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

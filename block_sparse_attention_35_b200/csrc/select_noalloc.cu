@@ -75,10 +75,10 @@ extern "C" PBSA_API int pbsa_select_blocks_noalloc(const pbsa_config* cfg, const
     float* kbar = reinterpret_cast<float*>(static_cast<char*>(scratch) + key_off);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     cudaError_t e = pbsa::launch_pool(g, static_cast<const __nv_bfloat16*>(q), q_frames,
-                                      static_cast<const __nv_bfloat16*>(k_local), local_frames, ring_head,
+                                      static_cast<const __nv_bfloat16*>(k_local), ring_head, local_frames,
                                       qbar, kbar, st);
     if (e != cudaSuccess) return pbsa::api_cuda_fail(e, "pool kernel launch");
-    e = pbsa::launch_score_topk(g, qbar, kbar, q_frames * g.nbf, local_frames * g.nbf, k, idx, idx_stride,
+    e = pbsa::launch_score_topk(g, qbar, kbar, ring_head, q_frames * g.nbf, local_frames * g.nbf, k, idx, idx_stride,
                                 cnt, scores, st);
     if (e != cudaSuccess) return pbsa::api_cuda_fail(e, "score/top-k kernel launch");
     return PBSA_OK;

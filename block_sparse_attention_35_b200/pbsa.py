@@ -88,6 +88,8 @@ def _load():
         "pbsa_cache_update": (I, [C, P, P, I, I, P, I, I, P, P, P, P, P, P, P, P,
                                   ctypes.c_size_t, P]),
         "pbsa_wait_selftest": (I, [P, ctypes.c_longlong, P]),
+        "pbsa_pool_keys": (I, [C, P, I, I, P, P]),
+        "pbsa_select_blocks_pooled": (I, [C, P, I, P, I, I, P, I, P, P, P, ctypes.c_size_t, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -214,6 +216,23 @@ def pbsa_cache_update(cfg, k_local, v_local, local_frames, ring_head, mass_local
 
 def pbsa_wait_selftest(status, timeout_ns: int, stream=None):
     _check(_lib.pbsa_wait_selftest(_ptr(status), int(timeout_ns), _stream(stream)))
+
+
+def pbsa_pool_keys(cfg, k_local, first_slot, n_frames, kbar, stream=None):
+    """Pools the key blocks of ring slots first_slot.. (n_frames, mod W) into kbar
+    [B, H, W*NB_f, D] fp32 (row = slot * NB_f + block)."""
+    _check(_lib.pbsa_pool_keys(_cfg(cfg), _ptr(k_local), first_slot, n_frames, _ptr(kbar),
+                               _stream(stream)))
+
+
+def pbsa_select_blocks_pooled(cfg, q, q_frames, kbar, local_frames, ring_head, idx, idx_stride,
+                              cnt, scores, workspace, stream=None):
+    """Block selection with the window's key means read from kbar (see pbsa_pool_keys)."""
+    _check(_lib.pbsa_select_blocks_pooled(
+        _cfg(cfg), _ptr(q), q_frames, _ptr(kbar), local_frames, ring_head, _ptr(idx),
+        idx_stride, _ptr(cnt), _ptr(scores), _ptr(workspace),
+        0 if workspace is None else workspace.numel() * workspace.element_size(),
+        _stream(stream)))
 
 
 def pbsa_select_blocks_noalloc(cfg, q, q_frames, k_local, local_frames, ring_head, idx,

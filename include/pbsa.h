@@ -176,6 +176,31 @@ PBSA_API int pbsa_select_blocks_noalloc(const pbsa_config* cfg, const void* q, i
                                         float* scores, void* stream);
 
 /*
+ * Key-mean cache (project page, kernel features: the KV cache is managed by the kernels; a
+ * reading, not a stated feature: a window block never changes while it is cached, so its
+ * pooled key can be computed once, when its frame is appended).  The paper has no separate
+ * call for this.
+ *
+ * pbsa_pool_keys: mean over the valid tokens of every 1x8x8 block of the n_frames frames in
+ * ring slots first_slot, first_slot+1, ... (mod W) of k_local [B, W*T_f, H, D] bf16, written
+ * to kbar [B, H, W*NB_f, D] fp32 at row (slot * NB_f + block) - the layout
+ * pbsa_select_blocks_pooled reads.  Rows of other slots are left as they are.  kbar is
+ * caller-owned device memory; no workspace.  PBSA_ERR_ARG on a bad slot/frame count.
+ *
+ * pbsa_select_blocks_pooled: pbsa_select_blocks with the window's key means taken from kbar
+ * (every slot of the window must have been pooled since its frame was written) instead of
+ * being recomputed from k_local: only the chunk's queries are pooled.  Same outputs and
+ * errors as pbsa_select_blocks; workspace >= B*H*q_frames*NB_f*D*4 bytes (256-aligned),
+ * not needed when every block is selected and scores is NULL.
+ */
+PBSA_API int pbsa_pool_keys(const pbsa_config* cfg, const void* k_local, int first_slot, int n_frames,
+                            float* kbar, void* stream);
+PBSA_API int pbsa_select_blocks_pooled(const pbsa_config* cfg, const void* q, int q_frames,
+                                       const float* kbar, int local_frames, int ring_head,
+                                       int32_t* idx, int idx_stride, int32_t* cnt, float* scores,
+                                       void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * PBSA forward.  (pith.science abstract; project page call attn(query, key_persistent,
  * value_persistent, key_local, value_local).)
  *
