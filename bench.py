@@ -287,8 +287,8 @@ def step(a, q, dout, ev=None):
 
 
 def kernels_per_step(with_bwd):
-    # pool, score/top-k, forward, [delta, dK/dV, dQ], merge rank, merge copy
-    return 5 + (3 if with_bwd else 0)
+    # pool, score/top-k, forward, [delta, dQ + dK/dV grid], merge rank, merge copy
+    return 5 + (2 if with_bwd else 0)
 
 
 def bwd_available(dev):
@@ -357,7 +357,7 @@ def run_ours(args, ws, rank, local):
         bwd_avg = sum(bwd_ms) / len(bwd_ms)
         bwd_ach = (sum(bwd_flops) / len(bwd_flops)) / (bwd_avg * 1e-3) / 1e12
         if bwd_avg > fwd_avg:
-            dominant = {"kernel": "attn_bwd (delta + dK/dV + dQ)", "achieved": bwd_ach, "ms": bwd_avg}
+            dominant = {"kernel": "attn_bwd (delta + dQ/dK/dV grid)", "achieved": bwd_ach, "ms": bwd_avg}
     traffic = None
     tfile = os.path.join(ROOT, "profiles", "traffic.json")
     if os.path.exists(tfile):

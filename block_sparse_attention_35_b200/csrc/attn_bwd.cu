@@ -5,7 +5,8 @@
 //   P  = exp(S - lse) with S = Q K^T / sqrt(D)   (recomputed from the forward's lse)
 //   dV = P^T dO,   dP = dO V^T,   Delta = rowsum(dO * O),   dS = P * (dP - Delta)
 //   dQ = dS K / sqrt(D),   dK = dS^T Q / sqrt(D)
-// Deterministic, no atomics, three kernels:
+// Deterministic, no atomics, two launches: delta_kernel, then one grid whose first CTAs are
+// the dQ part and the rest the dK/dV part (bwd_kernel):
 //  1. delta_kernel: Delta per query row (one pass over O and dO).
 //  2. dkdv_kernel: one CTA per key tile (128 keys: 16 compacted 8-row groups of the
 //     persistent slots, or a pair of local blocks); it loops over the query tiles that
@@ -143,14 +144,19 @@ __host__ __device__ inline DkdvPlan dkdv_plan(int D, int S, int n_qt) {
     return p;
 }
 
-struct DkdvKernelArgs {
+// Arguments of the backward launch: dQ CTAs and dK/dV CTAs share one grid (see bwd_kernel).
+struct BwdKernelArgs {
     BwdArgs a;
-    int n_pt_max;  // persistent key tiles per (b, h) in the grid
+    int n_pt_max;  // persistent key tiles per (b, h) of the dK/dV part
     int n_qt;      // query tiles per (b, h)
+    int ucap;      // capacity of a query tile's local-block union
+    int n_dq_x;    // dQ CTAs per (b, h): query tiles
+    int n_kd_x;    // dK/dV CTAs per (b, h): persistent + local key tiles
 };
 
+// dK/dV of key tile cta_x of head h, batch b (body of bwd_kernel's dK/dV CTAs).
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1) dkdv_kernel(const __grid_constant__ DkdvKernelArgs ka) {
+__device__ __forceinline__ void dkdv_body(const BwdKernelArgs& ka, const int cta_x, const int h, const int b) {
     constexpr int NH = D / 64;
     constexpr uint32_t TILE = NH * kHalf;
     constexpr uint32_t kTmS = 0, kTmP = 128, kTmDV = 256, kTmDK = 256 + D;
@@ -174,13 +180,13 @@ __global__ void __launch_bounds__(kThreads, 1) dkdv_kernel(const __grid_constant
     int* misc = reinterpret_cast<int*>(sm + PL.misc);
     volatile int* abort_flag = misc + 1;
 
-    const int h = blockIdx.y, b = blockIdx.z, bh = b * g.H + h;
+    const int bh = b * g.H + h;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int qb_total = a.q_frames * g.nbf;
     const int nq = a.q_frames * g.tf;
     const int nl = a.local_frames * g.nbf;
-    const bool pers_tile = (int)blockIdx.x < ka.n_pt_max;
-    const int tile = pers_tile ? blockIdx.x : blockIdx.x - ka.n_pt_max;
+    const bool pers_tile = cta_x < ka.n_pt_max;
+    const int tile = pers_tile ? cta_x : cta_x - ka.n_pt_max;
 
     uint64_t* kv_full = &bars[0];      // K and V tiles of this CTA (once)
     uint64_t* qd_full = &bars[1];      // [kNst] Q + dO + lse/Delta of a query tile
@@ -539,13 +545,10 @@ __host__ __device__ inline DqPlan dq_plan(int D, int S, int ucap) {
     return p;
 }
 
-struct DqKernelArgs {
-    BwdArgs a;
-    int ucap;
-};
 
+// dQ of query tile `tile` of head h, batch b (body of bwd_kernel's dQ CTAs).
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__ DqKernelArgs ka) {
+__device__ __forceinline__ void dq_body(const BwdKernelArgs& ka, const int tile, const int h, const int b) {
     constexpr int NH = D / 64;
     constexpr uint32_t TILE = NH * kHalf;
     constexpr uint32_t kTmS = 0, kTmP = 128, kTmQ = 256;
@@ -576,7 +579,7 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
     uint64_t* dq_done = &bars[9];
     uint64_t* drain = &bars[10];
 
-    const int tile = blockIdx.x, h = blockIdx.y, b = blockIdx.z, bh = b * g.H + h;
+    const int bh = b * g.H + h;
     const int qb_total = a.q_frames * g.nbf;
     const int nq = a.q_frames * g.tf;
     const int qb0 = 2 * tile;
@@ -842,6 +845,25 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
     }
 }
 
+// One grid for both gradient kernels, dQ CTAs first: they are the long ones (a query tile
+// against its whole key stream), so the many short dK/dV CTAs that follow fill the SMs the
+// last dQ wave leaves idle instead of starting after it.  The two parts are independent
+// (they only read the forward's tensors and Delta and write different outputs).
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant__ BwdKernelArgs ka) {
+    const int H = ka.a.g.H;
+    const int n_dq = ka.n_dq_x * H * ka.a.g.B;
+    int i = blockIdx.x;
+    if (i < n_dq) {
+        const int r = i / ka.n_dq_x;
+        dq_body<D>(ka, i % ka.n_dq_x, r % H, r / H);
+    } else {
+        i -= n_dq;
+        const int r = i / ka.n_kd_x;
+        dkdv_body<D>(ka, i % ka.n_kd_x, r % H, r / H);
+    }
+}
+
 template <class K, class A>
 cudaError_t launch_k(K kernel, const A& args, dim3 grid, size_t smem, cudaStream_t st) {
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -869,23 +891,19 @@ cudaError_t launch_attn_bwd(const BwdArgs& a, cudaStream_t st) {
     if (e != cudaSuccess) return e;
 
     const int qb_total = a.q_frames * g.nbf;
-    DkdvKernelArgs kd;
-    kd.a = a;
-    kd.n_pt_max = (g.S * 8 + 15) / 16;
-    kd.n_qt = (qb_total + 1) / 2;
-    const int n_lt = (a.local_frames * g.nbf + 1) / 2;
-    const size_t smem_kd = attn_bwd_smem_bytes(g, a.q_frames, a.ucap);
-    dim3 grid_kd(kd.n_pt_max + n_lt, g.H, g.B);
-    e = g.D == 128 ? launch_k(dkdv_kernel<128>, kd, grid_kd, smem_kd, st)
-                   : launch_k(dkdv_kernel<64>, kd, grid_kd, smem_kd, st);
-    if (e != cudaSuccess) return e;
-
-    DqKernelArgs kq;
-    kq.a = a;
-    kq.ucap = a.ucap;
-    dim3 grid_q((qb_total + 1) / 2, g.H, g.B);
-    return g.D == 128 ? launch_k(dq_kernel<128>, kq, grid_q, smem_kd, st)
-                      : launch_k(dq_kernel<64>, kq, grid_q, smem_kd, st);
+    BwdKernelArgs ka;
+    ka.a = a;
+    ka.n_pt_max = (g.S * 8 + 15) / 16;
+    ka.n_qt = (qb_total + 1) / 2;
+    ka.ucap = a.ucap;
+    ka.n_dq_x = (qb_total + 1) / 2;
+    ka.n_kd_x = ka.n_pt_max + (a.local_frames * g.nbf + 1) / 2;
+    const size_t smem = attn_bwd_smem_bytes(g, a.q_frames, a.ucap);
+    const long long ctas = (long long)(ka.n_dq_x + ka.n_kd_x) * g.H * g.B;
+    if (ctas > 0x7fffffffll) return cudaErrorInvalidConfiguration;
+    dim3 grid((unsigned)ctas);
+    return g.D == 128 ? launch_k(bwd_kernel<128>, ka, grid, smem, st)
+                      : launch_k(bwd_kernel<64>, ka, grid, smem, st);
 }
 
 }  // namespace pbsa
