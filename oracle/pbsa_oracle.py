@@ -40,7 +40,7 @@ import numpy as np
 
 __all__ = ["frame_blocks", "topk_count", "pool_blocks", "block_scores", "select_topk",
            "select_blocks", "attend_rows", "attn_fwd", "cache_update", "attn_bwd",
-           "slot_capacity", "n_slots"]
+           "slot_capacity", "n_slots", "evict_count", "DecodeState", "decode_step"]
 
 
 # ---------------------------------------------------------------------------------------
@@ -390,3 +390,104 @@ def attn_bwd(q, k_pers, v_pers, pers_len, k_win, v_win, idx, dO, frame_h, frame_
                 np.add.at(dKw[b, :, h, :], ltok, dk[npers:])
                 np.add.at(dVw[b, :, h, :], ltok, dv[npers:])
     return dQ, dKp, dVp, dKw, dVw
+
+
+# ---------------------------------------------------------------------------------------
+# The t=0 KV pass of one chunk, end to end (pith.science page, algorithm fragment in the
+# reference list: the cache pass "applies PBSA with top-k and updates P and L"; abstract:
+# the persistent blocks are preserved and updated as the window slides)
+# ---------------------------------------------------------------------------------------
+def evict_count(frames_in_window: int, chunk_frames: int, window_frames: int) -> int:
+    """Frames that leave the window after a chunk's pass so that the next chunk fits.
+
+    Reading: the window holds window_frames frames including the current chunk; after the
+    pass, if frames_in_window + chunk_frames > window_frames, the oldest
+    frames_in_window + chunk_frames - window_frames frames are evicted (for a 6-frame
+    window and 3-frame chunks: nothing after chunk 0, then 3 frames after every chunk)."""
+    return max(0, frames_in_window + chunk_frames - window_frames)
+
+
+class DecodeState:
+    """Cache state between chunks, in the oracle's own plain layout (one batch item list
+    entry per array axis as in the other oracle functions):
+
+      win_k, win_v   [B, frames * T_f, H, D] window tokens, oldest frame first
+      win_mass       [B, H, frames * NB_f]   accumulated mass of every window block
+      k_pers, v_pers [B, H, S, 64, D]; pers_len, pers_src [B, H, S]; pers_score [B, H, S]
+      first_frame_global: global frame number of the oldest window frame
+    """
+
+    def __init__(self, win_k, win_v, win_mass, k_pers, v_pers, pers_len, pers_score, pers_src,
+                 first_frame_global=0):
+        self.win_k = np.asarray(win_k, np.float64)
+        self.win_v = np.asarray(win_v, np.float64)
+        self.win_mass = np.asarray(win_mass, np.float64)
+        self.k_pers = np.asarray(k_pers, np.float64)
+        self.v_pers = np.asarray(v_pers, np.float64)
+        self.pers_len = np.asarray(pers_len, np.int64)
+        self.pers_score = np.asarray(pers_score, np.float64)
+        self.pers_src = np.asarray(pers_src, np.int64)
+        self.first_frame_global = int(first_frame_global)
+
+    @classmethod
+    def empty(cls, B, H, D, S, frame_h, frame_w, bh=8, bw=8):
+        """A rollout's start: empty window, empty persistent cache."""
+        return cls(np.zeros((B, 0, H, D)), np.zeros((B, 0, H, D)), np.zeros((B, H, 0)),
+                   np.zeros((B, H, S, bh * bw, D)), np.zeros((B, H, S, bh * bw, D)),
+                   np.zeros((B, H, S), np.int64), np.zeros((B, H, S)),
+                   np.full((B, H, S), -1, np.int64))
+
+
+def decode_step(state: DecodeState, q, k_chunk, v_chunk, ratio, window_frames, frame_h,
+                frame_w, use_sparse=True, idx=None, bh=8, bw=8):
+    """One chunk's cache pass, in the order of the algorithm fragment:
+
+      1. the chunk's frames join the window (reading: before its attention, so the window
+         includes the current chunk);
+      2. top-k block selection over the window (select_blocks), unless `idx` is given
+         (a caller may pass another implementation's selection to compare the rest of the
+         step on equal terms);
+      3. the PBSA forward with block mass (attn_fwd);
+      4. the masses are accumulated: every window block and every persistent slot adds the
+         probability mass it received in this pass (reading: per head, never decayed);
+      5. slide: evict_count(frames, chunk frames, window_frames) oldest frames leave the
+         window, and their blocks are merged into the persistent cache by accumulated mass
+         (cache_update); the evicted blocks' masses leave with them.
+
+    Returns (new_state, out) with out = dict(idx, scores, O, lse, mass_pers, mass_local,
+    n_evict, updates).  The input state is not modified.
+    """
+    blocks = frame_blocks(frame_h, frame_w, bh, bw)
+    nbf = len(blocks)
+    tf = frame_h * frame_w
+    chunk_frames = np.asarray(k_chunk).shape[1] // tf
+    frames = state.win_k.shape[1] // tf + chunk_frames
+    if frames > window_frames:
+        raise ValueError("the window has no room for the chunk")
+    win_k = np.concatenate([state.win_k, np.asarray(k_chunk, np.float64)], axis=1)
+    win_v = np.concatenate([state.win_v, np.asarray(v_chunk, np.float64)], axis=1)
+    B, H = state.pers_len.shape[:2]
+    win_mass = np.concatenate([state.win_mass, np.zeros((B, H, chunk_frames * nbf))], axis=2)
+    scores = None
+    if idx is None:
+        idx, scores = select_blocks(q, win_k, frame_h, frame_w, ratio, use_sparse, bh, bw)
+    O, lse, mass_pers, mass_local = attn_fwd(q, state.k_pers, state.v_pers, state.pers_len,
+                                             win_k, win_v, idx, frame_h, frame_w, bh, bw)
+    win_mass = win_mass + mass_local
+    pers_score = state.pers_score + mass_pers
+    n_ev = evict_count(frames, chunk_frames, window_frames)
+    out = dict(idx=idx, scores=scores, O=O, lse=lse, mass_pers=mass_pers,
+               mass_local=mass_local, n_evict=n_ev, updates=[[[] for _ in range(H)] for _ in range(B)],
+               pers_score_before_merge=pers_score, win_mass_before_merge=win_mass)
+    if n_ev == 0:
+        new = DecodeState(win_k, win_v, win_mass, state.k_pers, state.v_pers, state.pers_len,
+                          pers_score, state.pers_src, state.first_frame_global)
+        return new, out
+    r = cache_update(state.k_pers, state.v_pers, state.pers_len, pers_score, state.pers_src,
+                     win_k, win_v, win_mass, n_ev, state.first_frame_global, frame_h, frame_w,
+                     bh, bw)
+    out["updates"] = r["updates"]
+    new = DecodeState(win_k[:, n_ev * tf:], win_v[:, n_ev * tf:], win_mass[:, :, n_ev * nbf:],
+                      r["k_pers"], r["v_pers"], r["pers_len"], r["pers_score"], r["pers_src"],
+                      state.first_frame_global + n_ev)
+    return new, out

@@ -476,3 +476,100 @@ def test_dense_cache_mode_forward_is_dense_attention_over_the_window():
             want = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt)[0, 0].numpy()
             assert np.allclose(O[b, :, h], want, rtol=0, atol=1e-12)
     assert mp.size == 0
+
+
+# ------------------------------------------------------------- slot count, multi-chunk
+def test_n_slots_whole_frames_and_token_budget():
+    # whole frames: frames x blocks per frame (16x16 has 4 blocks, 30x52 has 28)
+    assert orc.n_slots(256, 16, 16) == 4
+    assert orc.n_slots(512, 16, 16) == 8
+    assert orc.n_slots(9360, 30, 52) == 168
+    assert orc.n_slots(4680, 30, 52) == 84
+    # otherwise the token budget in 64-row slots, rounded up
+    assert orc.n_slots(64, 16, 16) == 1
+    assert orc.n_slots(100, 16, 16) == 2
+    assert orc.n_slots(129, 16, 16) == 3
+    assert orc.n_slots(1000, 30, 52) == 16
+
+
+@pytest.mark.parametrize("W,E,want", [(6, 3, [0, 3, 3, 3, 3]), (4, 1, [0, 0, 0, 1, 1, 1]),
+                                      (5, 2, [0, 1, 2, 2, 2]), (2, 2, [2, 2, 2])])
+def test_evict_count_hand_sequences(W, E, want):
+    frames, got = 0, []
+    for _ in want:
+        frames += E            # the chunk joins the window
+        assert frames <= W
+        ev = orc.evict_count(frames, E, W)
+        got.append(ev)
+        frames -= ev
+    assert got == want
+
+
+def _hand_rollout_inputs():
+    """Frames of 8x16 tokens (two 8x8 blocks), D = 4, one batch item and head.  Every query
+    row is (2, 0, 0, 0); keys are zero except frame 2's block 1, whose tokens are
+    (10, 0, 0, 0).  So a zero key scores logit 0, a hot key 2 * 10 / sqrt(4) = 10."""
+    fh, fw, D = 8, 16, 4
+    tf = fh * fw
+    rng = np.random.default_rng(5)
+    chunks = []
+    for c in range(4):
+        q = np.zeros((1, tf, 1, D))
+        q[..., 0] = 2.0
+        k = np.zeros((1, tf, 1, D))
+        if c == 2:
+            k[0, orc.frame_blocks(fh, fw)[1], 0, 0] = 10.0
+        v = rng.standard_normal((1, tf, 1, D))
+        chunks.append((q, k, v))
+    return fh, fw, D, chunks
+
+
+def test_decode_step_hand_rollout_fill_admit_and_turnover():
+    """Window of 2 frames, 1-frame chunks, 2 persistent slots, ratio 0.5, values worked out
+    by hand: uniform attention while every key is zero, then a hot block that takes almost
+    all the probability and, two passes later, displaces the weaker slot."""
+    fh, fw, D, chunks = _hand_rollout_inputs()
+    st = orc.DecodeState.empty(1, 1, D, 2, fh, fw)
+    outs = []
+    for q, k, v in chunks:
+        st, o = orc.decode_step(st, q, k, v, 0.5, 2, fh, fw)
+        outs.append((st, o))
+    Z = 192.0 + 64.0 * math.exp(10.0)
+    a, hot = 8192.0 / Z, 8192.0 * math.exp(10.0) / Z     # per-pass mass of a cold / hot block
+    # chunk 0: window [f0]; k = ceil(0.5 * 2) = 1 -> block 0 (tie to the lower id); every
+    # row spreads over its 64 keys, so block 0 gets 128 rows x 1 and O = mean of its values
+    st0, o0 = outs[0]
+    assert o0["n_evict"] == 0 and o0["idx"].tolist() == [[[[0], [0]]]]
+    assert np.allclose(o0["mass_local"][0, 0], [128.0, 0.0], rtol=0, atol=1e-12)
+    vmean = chunks[0][2][0, orc.frame_blocks(fh, fw)[0], 0].mean(axis=0)
+    assert np.allclose(o0["O"][0, :, 0], vmean, rtol=0, atol=1e-12)
+    assert (st0.pers_len == 0).all()
+    # chunk 1: window [f0, f1]; k = 2 -> blocks 0, 1 (all ties); 128 keys per row, 64 each;
+    # accumulated f0 masses 192, 64; evict f0 into the empty cache in id order
+    st1, o1 = outs[1]
+    assert o1["idx"].tolist() == [[[[0, 1], [0, 1]]]]
+    assert np.allclose(o1["mass_local"][0, 0], [64, 64, 0, 0], rtol=0, atol=1e-12)
+    assert o1["n_evict"] == 1 and o1["updates"][0][0] == [(0, 0), (1, 1)]
+    assert st1.pers_len.tolist() == [[[64, 64]]]
+    assert np.allclose(st1.pers_score[0, 0], [192.0, 64.0], rtol=0, atol=1e-12)
+    assert st1.pers_src.tolist() == [[[0, 1]]]
+    assert np.allclose(st1.win_mass[0, 0], [0.0, 0.0]) and st1.first_frame_global == 1
+    # chunk 2: window [f1, f2]; the hot block (id 3) scores 10, the rest 0 -> {0, 3};
+    # keys per row: 128 slot rows + f1 block 0 (logit 0) + the hot block (logit 10)
+    st2, o2 = outs[2]
+    assert o2["idx"].tolist() == [[[[0, 3], [0, 3]]]]
+    assert np.allclose(o2["mass_pers"][0, 0], [a, a], rtol=1e-12, atol=0)
+    assert np.allclose(o2["mass_local"][0, 0], [a, 0.0, 0.0, hot], rtol=1e-12, atol=1e-15)
+    assert o2["n_evict"] == 1 and o2["updates"][0][0] == []     # f1's blocks lose to both slots
+    assert np.allclose(st2.pers_score[0, 0], [192 + a, 64 + a], rtol=1e-12, atol=0)
+    assert np.allclose(st2.win_mass[0, 0], [0.0, hot], rtol=1e-12, atol=1e-15)
+    # chunk 3: window [f2, f3]; the hot block is now id 1 -> {0, 1}; f2's block 1 has two
+    # passes of mass (2 hot > 192 + 2a) and displaces slot 1 (64 + 2a)
+    st3, o3 = outs[3]
+    assert o3["idx"].tolist() == [[[[0, 1], [0, 1]]]]
+    assert o3["n_evict"] == 1 and o3["updates"][0][0] == [(1, 1)]
+    assert np.allclose(st3.pers_score[0, 0], [192 + 2 * a, 2 * hot], rtol=1e-12, atol=0)
+    assert st3.pers_src.tolist() == [[[0, 2 * 2 + 1]]]     # global frame 2, block 1
+    assert st3.pers_len.tolist() == [[[64, 64]]]
+    assert (st3.k_pers[0, 0, 1, :, 0] == 10.0).all() and (st3.k_pers[0, 0, 1, :, 1:] == 0).all()
+    assert st3.first_frame_global == 3 and st3.win_k.shape[1] == 128
