@@ -5,25 +5,27 @@
 //   P  = exp(S - lse) with S = Q K^T / sqrt(D)   (recomputed from the forward's lse)
 //   dV = P^T dO,   dP = dO V^T,   Delta = rowsum(dO * O),   dS = P * (dP - Delta)
 //   dQ = dS K / sqrt(D),   dK = dS^T Q / sqrt(D)
-// Deterministic, no atomics, two launches: delta_kernel, then one grid whose first CTAs are
-// the dQ part and the rest the dK/dV part (bwd_kernel):
+// Deterministic, no atomics, two launches: delta_kernel, then bwd_kernel, one grid whose
+// first CTAs compute dQ and whose other CTAs compute dK/dV:
 //  1. delta_kernel: Delta per query row (one pass over O and dO).
-//  2. dkdv_kernel: one CTA per key tile (128 keys: 16 compacted 8-row groups of the
-//     persistent slots, or a pair of local blocks); it loops over the query tiles that
-//     attend to those keys (all of them for persistent keys; for local blocks the query
-//     tiles whose query blocks selected either block).  S^T = K Q^T and dP^T = V dO^T land
-//     in TMEM (lanes = keys); 16 element warps (a key-row quarter and 32 query columns
-//     each) form P^T and dS^T, write them as bf16 back over S^T / dP^T, and two TS MMAs
-//     accumulate dV += P^T dO and dK += dS^T Q in TMEM (dO and Q tiles read MN-major from
-//     shared memory).
-//  3. dq_kernel: one CTA per query tile (the forward's tiling); per key tile S = Q K^T and
-//     dP = dO V^T in TMEM, the element warps (a query-row quarter and 32 key columns each)
-//     form dS, write it as bf16 over S, and a TS MMA accumulates dQ += dS K (K read
-//     MN-major).
-// Warp roles in 2 and 3: warps 0-15 elementwise (P, dS), warp 16 TMA producer, warp 17 MMA.
-// The MMA thread issues the next tile's S / dP right after the current tile's gradient
-// MMAs (the tensor pipe runs them in issue order), so only the element warps' work on a
-// tile leaves the pipe idle.
+//  2. bwd_kernel, dK/dV CTAs (dkdv_body): one CTA per key tile (128 keys: 16 compacted
+//     8-row groups of the persistent slots, or a pair of local blocks); it loops over the
+//     query tiles that attend to those keys (all of them for persistent keys; for local
+//     blocks the query tiles whose query blocks selected either block).  S^T = K Q^T and
+//     dP^T = V dO^T land in TMEM (lanes = keys); 16 element warps (a key-row quarter and 32
+//     query columns each) form P^T and dS^T, write them as bf16 back over S^T / dP^T, and
+//     two TS MMAs accumulate dV += P^T dO and dK += dS^T Q in TMEM (dO and Q tiles read
+//     MN-major from shared memory).
+//  3. bwd_kernel, dQ CTAs (dq_body): one CTA per query tile (the forward's tiling); per key
+//     tile S = Q K^T and dP = dO V^T in TMEM, the element warps (a query-row quarter and 32
+//     key columns each) form dS, write it as bf16 over S, and a TS MMA accumulates
+//     dQ += dS K (K read MN-major).
+// Warp roles in both parts: warps 0-15 elementwise (P, dS), warp 16 TMA producer, warp 17
+// MMA.  The MMA thread issues the next tile's S / dP right after the current tile's
+// gradient MMAs (the tensor pipe runs them in issue order), so only the element warps'
+// work on a tile leaves the pipe idle.  Persistent slots of any length 1..64 are streamed
+// as ceil(len / 8) groups; rows of a partial last group past the slot's length are masked
+// (P and dS exactly zero), so they only need to hold finite values.
 #include <cuda_bf16.h>
 #include <math_constants.h>
 
@@ -92,8 +94,10 @@ __global__ void __launch_bounds__(256) delta_kernel(const __nv_bfloat16* __restr
 }
 
 // --------------------------------------------------------- persistent group table
-// Builds, with one warp, the compacted list of the occupied slots' 8-row groups: row
-// index of each group in the [B*H*S*64, D] slot store.  Returns the group count.
+// Builds, with one warp, the compacted list of the occupied slots' 8-row groups
+// (ceil(len / 8) per slot): the first row of each group in the [B*H*S*64, D] slot store,
+// with the group's valid-row count & 7 in the low 3 bits (0 = all 8 rows valid; only a
+// slot's last group can be partial).  Returns the group count.
 __device__ int build_groups(const int32_t* pers_len, int bh, int S, int32_t* grp_row,
                             int32_t* status) {
     const int lane = threadIdx.x & 31;
@@ -101,11 +105,11 @@ __device__ int build_groups(const int32_t* pers_len, int bh, int S, int32_t* grp
     for (int s0 = 0; s0 < S; s0 += 32) {
         const int s = s0 + lane;
         int len = (s < S) ? pers_len[(size_t)bh * S + s] : 0;
-        if (len < 0 || len > 64 || (len & 7)) {
+        if (len < 0 || len > 64) {
             set_status(status, PBSA_ERR_DEVICE_CHECK);
             len = 0;
         }
-        const int ng = len >> 3;
+        const int ng = (len + 7) >> 3;
         int inc = ng;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -113,10 +117,17 @@ __device__ int build_groups(const int32_t* pers_len, int bh, int S, int32_t* grp
             if (lane >= o) inc += v;
         }
         const int gstart = run + inc - ng;
-        for (int i = 0; i < ng; ++i) grp_row[gstart + i] = ((bh * S) + s) * 64 + 8 * i;
+        for (int i = 0; i < ng; ++i)
+            grp_row[gstart + i] = (((bh * S) + s) * 64 + 8 * i) | (min(8, len - 8 * i) & 7);
         run += __shfl_sync(0xffffffffu, inc, 31);
     }
     return run;
+}
+
+// Valid rows (1..8) of a group-table entry.
+__device__ __forceinline__ int group_rows(int32_t entry) {
+    const int nv = entry & 7;
+    return nv ? nv : 8;
 }
 
 constexpr int B_COUNT = 12;  // mbarrier slots reserved per CTA
@@ -407,7 +418,8 @@ __device__ __forceinline__ void dkdv_body(const BwdKernelArgs& ka, const int cta
         bool key_valid;
         int kbr = 0;
         if (pers_tile) {
-            key_valid = tile * 16 + (r >> 3) < G;
+            const int gi = tile * 16 + (r >> 3);
+            key_valid = gi < G && (r & 7) < group_rows(grp_row[gi]);
         } else {
             kbr = r >> 6;
             const int L = kbr ? L1 : L0;
@@ -450,7 +462,7 @@ __device__ __forceinline__ void dkdv_body(const BwdKernelArgs& ka, const int cta
 #pragma unroll
                     for (int u = 0; u < 4; ++u) {
                         p[u] = sel ? fast_exp2(__uint_as_float(sv[4 * e4 + u]) * sl2 - ls[u]) : 0.f;
-                        d[u] = p[u] * (__uint_as_float(pv[4 * e4 + u]) - ds[u]);
+                        d[u] = sel ? p[u] * (__uint_as_float(pv[4 * e4 + u]) - ds[u]) : 0.f;
                     }
                     pk[8 * sc + 2 * e4] = pack_bf16x2(p[0], p[1]);
                     pk[8 * sc + 2 * e4 + 1] = pack_bf16x2(p[2], p[3]);
@@ -476,7 +488,7 @@ __device__ __forceinline__ void dkdv_body(const BwdKernelArgs& ka, const int cta
             float* dv_row = nullptr;
             if (key_valid) {
                 if (pers_tile) {
-                    const size_t row = (size_t)grp_row[tile * 16 + (r >> 3)] + (r & 7);
+                    const size_t row = (size_t)(grp_row[tile * 16 + (r >> 3)] & ~7) + (r & 7);
                     dk_row = a.dk_pers + row * D;
                     dv_row = a.dv_pers + row * D;
                 } else {
@@ -668,7 +680,7 @@ __device__ __forceinline__ void dq_body(const BwdKernelArgs& ka, const int tile,
                 mbar_arrive_expect_tx(&v_full[st], TILE);
                 if (it < n_pt) {
                     for (int c = 0; c < 16; ++c) {
-                        const int row = grp_row[min(it * 16 + c, G - 1)];
+                        const int row = grp_row[min(it * 16 + c, G - 1)] & ~7;
                         for (int hh = 0; hh < NH; ++hh) {
                             tma_load_2d(dk + hh * kHalf + c * 1024, &a.tm_kp, &k_full[st], hh * 64, row);
                             tma_load_2d(dv + hh * kHalf + c * 1024, &a.tm_vp, &v_full[st], hh * 64, row);
@@ -765,8 +777,16 @@ __device__ __forceinline__ void dq_body(const BwdKernelArgs& ka, const int tile,
             // valid-column mask of this warp's 32 key columns
             uint32_t vmask;
             if (it < n_pt) {
-                const int nvc = min(128, 8 * (G - 16 * it)) - c0;   // valid persistent columns left
-                vmask = nvc >= kCw ? 0xffffffffu : (nvc <= 0 ? 0u : ((1u << nvc) - 1u));
+                // the warp's 32 columns are groups 16 it + c0 / 8 .. + 3 of the stream
+                vmask = 0u;
+#pragma unroll
+                for (int gq = 0; gq < kCw / 8; ++gq) {
+                    const int gi = 16 * it + c0 / 8 + gq;
+                    if (gi < G) {
+                        const int nv = group_rows(grp_row[gi]);
+                        vmask |= (nv >= 8 ? 0xffu : ((1u << nv) - 1u)) << (8 * gq);
+                    }
+                }
             } else {
                 const int u = 2 * (it - n_pt) + kh;
                 const bool has = u < U;
@@ -797,8 +817,8 @@ __device__ __forceinline__ void dq_body(const BwdKernelArgs& ka, const int tile,
 #pragma unroll
                     for (int u = 0; u < 2; ++u) {
                         const bool valid = (vmask >> (16 * sc + e + u)) & 1u;
-                        const float p = valid ? fast_exp2(__uint_as_float(sv[e + u]) * sl2 - lse2) : 0.f;
-                        dsv[u] = p * (__uint_as_float(pv[e + u]) - dl);
+                        const float p = fast_exp2(__uint_as_float(sv[e + u]) * sl2 - lse2);
+                        dsv[u] = valid ? p * (__uint_as_float(pv[e + u]) - dl) : 0.f;
                     }
                     dk[8 * sc + e / 2] = pack_bf16x2(dsv[0], dsv[1]);
                 }

@@ -10,9 +10,11 @@
 // One CTA = four 8x8 query blocks of one (batch, head), split into two 128-row query tiles
 // ("sides" A and B, two blocks each, every block a 64-row 5-D TMA box; ragged edge blocks
 // are zero-filled on load and clipped on store).  Key tiles are 128 keys:
-//   * persistent tiles (shared by both sides): the occupied slots' valid rows compacted
-//     into a stream of 8-row groups (slot lengths are multiples of 8), 16 groups per tile,
-//     loaded as one 64-row TMA box wherever eight groups are contiguous rows (a full slot);
+//   * persistent tiles (shared by both sides): the occupied slots' rows compacted into a
+//     stream of 8-row groups (ceil(len / 8) groups per slot; the last group of a slot whose
+//     length is not a multiple of 8 is partly valid and its other rows are masked), 16
+//     groups per tile, loaded as one 64-row TMA box wherever eight groups are contiguous
+//     rows (a full slot);
 //   * local tiles (one side each): the union of that side's two selections, two 8x8 key
 //     blocks per tile; columns the row's query block did not select, or outside the frame,
 //     are masked.  A-tiles and B-tiles alternate in the stream.
@@ -53,11 +55,10 @@ constexpr int kThreads = 384;
 constexpr int kLaunchRegs = 168, kRegsIo = 104, kRegsSoftmax = 200;
 static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsIo <= kThreads * kLaunchRegs, "register split");
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr int kEmuPairs = 0;  // of every 4 exponential pairs, this many on the FMA pipe (measured: no gain)
 
 struct SmemPlan {
-    uint32_t q, k, v, grp_row, grp_seg, seg_slot, tile_end, tile_seg, uni_blk, uni_bits, lse_s,
-        bars, misc, total;
+    uint32_t q, k, v, grp_row, grp_seg, seg_slot, tile_end, tile_seg, tile_mask, uni_blk, uni_bits,
+        lse_s, bars, misc, total;
 };
 
 __host__ __device__ inline SmemPlan fwd_plan(int D, int S, int ucap) {
@@ -72,7 +73,8 @@ __host__ __device__ inline SmemPlan fwd_plan(int D, int S, int ucap) {
     p.seg_slot = p.grp_seg + 4u * 8u * S;
     p.tile_end = p.seg_slot + 4u * S;        // per persistent tile: groups that end a slot
     p.tile_seg = p.tile_end + 4u * n_pt_max; // per persistent tile: slot rank of group 0
-    p.uni_blk = p.tile_seg + 4u * n_pt_max;  // [2][ucap]
+    p.tile_mask = p.tile_seg + 4u * n_pt_max; // per persistent tile: 128-bit valid-column mask
+    p.uni_blk = p.tile_mask + 16u * n_pt_max; // [2][ucap]
     p.uni_bits = p.uni_blk + 8u * ucap;      // [2][ucap]
     p.lse_s = p.uni_bits + 8u * ucap;        // [2][128] row log-sum-exp (log2) for the mass
     p.bars = (p.lse_s + 2u * 128u * 4u + 7u) & ~7u;
@@ -110,40 +112,8 @@ __device__ __forceinline__ float2 ffma2(float2 a, float s, float m) {
     return make_float2(__uint_as_float(static_cast<uint32_t>(r)), __uint_as_float(static_cast<uint32_t>(r >> 32)));
 }
 
-__device__ __forceinline__ float2 fma2v(float2 a, float2 b, float2 c) {
-    float2 d;
-    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
-        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
-        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-        : "=f"(d.x), "=f"(d.y)
-        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
-    return d;
-}
-
-// 2^x on the FMA and integer pipes, for two values (x <= 9).  Cody-Waite style range
-// reduction: adding 1.5 * 2^23 rounds x to the nearest integer n (kept in the low mantissa
-// bits of y) and leaves f = x - n in [-1/2, 1/2]; 2^f is a degree-3 polynomial fitted here
-// for minimum relative error (max 7.5e-5, far below bf16 rounding); n is added to the
-// exponent field.  Inputs below -125 are clamped (the result is then about 2^-125).
-__device__ __forceinline__ float2 exp2_poly2(float2 x) {
-    constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
-    constexpr float c0 = 0.9999281167984009f, c1 = 0.6932609677314758f;
-    constexpr float c2 = 0.24261054396629333f, c3 = 0.05517132207751274f;
-    x.x = fmaxf(x.x, -125.0f);
-    x.y = fmaxf(x.y, -125.0f);
-    const float2 y = fma2v(x, make_float2(1.0f, 1.0f), make_float2(kMagic, kMagic));
-    const float2 t = fma2v(y, make_float2(1.0f, 1.0f), make_float2(-kMagic, -kMagic));
-    const float2 f = fma2v(t, make_float2(-1.0f, -1.0f), x);
-    float2 q = fma2v(make_float2(c3, c3), f, make_float2(c2, c2));
-    q = fma2v(q, f, make_float2(c1, c1));
-    q = fma2v(q, f, make_float2(c0, c0));
-    return make_float2(__uint_as_float(__float_as_uint(q.x) + (__float_as_uint(y.x) << 23)),
-                       __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(y.y) << 23)));
-}
-
-// exp_half<0, 0> plus the maximum of all 128 raw values, read before they are overwritten:
+// exp_half<0> plus the maximum of all 128 raw values, read before they are overwritten:
 // the ALU max work interleaves with the MUFU exponentials.
-template <int EMU>
 __device__ __forceinline__ float exp_half0_max(float (&x)[128], float sl2, float mu, float (&gs)[16]) {
     float mx[8];
 #pragma unroll
@@ -158,14 +128,8 @@ __device__ __forceinline__ float exp_half0_max(float (&x)[128], float sl2, float
         for (int pr = 0; pr < 4; ++pr) {
             const int c = 8 * gq + 2 * pr;
             const float2 q = ffma2(make_float2(x[c], x[c + 1]), sl2, mu);
-            if (pr >= 4 - EMU) {
-                const float2 e = exp2_poly2(q);
-                x[c] = e.x;
-                x[c + 1] = e.y;
-            } else {
-                x[c] = fast_exp2(q.x);
-                x[c + 1] = fast_exp2(q.y);
-            }
+            x[c] = fast_exp2(q.x);
+            x[c + 1] = fast_exp2(q.y);
         }
         gs[gq] = ((x[8 * gq + 0] + x[8 * gq + 1]) + (x[8 * gq + 2] + x[8 * gq + 3])) +
                  ((x[8 * gq + 4] + x[8 * gq + 5]) + (x[8 * gq + 6] + x[8 * gq + 7]));
@@ -174,9 +138,8 @@ __device__ __forceinline__ float exp_half0_max(float (&x)[128], float sl2, float
 }
 
 // p = 2^(x * sl2 - mu) over the 64 columns [64 H, 64 H + 64) of a row, in place, with their
-// 8-column group sums; EMU of the four pairs in each group go through exp2_poly2, the rest
-// through MUFU.
-template <int EMU, int H>
+// 8-column group sums.
+template <int H>
 __device__ __forceinline__ void exp_half(float (&x)[128], float sl2, float mu, float (&gs)[16]) {
 #pragma unroll
     for (int gq = 8 * H; gq < 8 * H + 8; ++gq) {
@@ -184,14 +147,8 @@ __device__ __forceinline__ void exp_half(float (&x)[128], float sl2, float mu, f
         for (int pr = 0; pr < 4; ++pr) {
             const int c = 8 * gq + 2 * pr;
             const float2 q = ffma2(make_float2(x[c], x[c + 1]), sl2, mu);
-            if (pr >= 4 - EMU) {
-                const float2 e = exp2_poly2(q);
-                x[c] = e.x;
-                x[c + 1] = e.y;
-            } else {
-                x[c] = fast_exp2(q.x);
-                x[c + 1] = fast_exp2(q.y);
-            }
+            x[c] = fast_exp2(q.x);
+            x[c + 1] = fast_exp2(q.y);
         }
         gs[gq] = ((x[8 * gq + 0] + x[8 * gq + 1]) + (x[8 * gq + 2] + x[8 * gq + 3])) +
                  ((x[8 * gq + 4] + x[8 * gq + 5]) + (x[8 * gq + 6] + x[8 * gq + 7]));
@@ -204,10 +161,6 @@ __device__ __forceinline__ uint64_t block_mask(bool sel, int hv, int wv) {
     const uint64_t rows = hv >= 8 ? ~0ull : ((1ull << (8 * hv)) - 1ull);
     const uint64_t cols = 0x0101010101010101ull * static_cast<uint64_t>((1u << wv) - 1u);
     return rows & cols;
-}
-
-__device__ __forceinline__ uint64_t prefix_mask(int n) {  // bits [0, n), n in [0, 64]
-    return n >= 64 ? ~0ull : ((1ull << n) - 1ull);
 }
 
 // Consumers of stream tile t: bit 0 = side A, bit 1 = side B; *lj = local tile index.
@@ -247,6 +200,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     int32_t* seg_slot = reinterpret_cast<int32_t*>(sm + P.seg_slot);
     uint32_t* tile_end = reinterpret_cast<uint32_t*>(sm + P.tile_end);
     int32_t* tile_seg = reinterpret_cast<int32_t*>(sm + P.tile_seg);
+    uint4* tile_mask = reinterpret_cast<uint4*>(sm + P.tile_mask);
     int32_t* uni_blk = reinterpret_cast<int32_t*>(sm + P.uni_blk);
     int32_t* uni_bits = reinterpret_cast<int32_t*>(sm + P.uni_bits);
     float* lse_s = reinterpret_cast<float*>(sm + P.lse_s);
@@ -286,16 +240,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     }
     if (warp == 10) tmem_alloc(reinterpret_cast<uint32_t*>(misc + M_TMEM), kTmCols);
     if (warp == 0) {
-        // compacted stream of the occupied slots' 8-row groups
+        // compacted stream of the occupied slots' 8-row groups; a group's entry is its first
+        // row in the slot store with (valid rows & 7) in the low 3 bits (0 = all 8 valid)
         int run = 0, occ = 0;
         for (int s0 = 0; s0 < S; s0 += 32) {
             const int s = s0 + lane;
             int len = (s < S) ? a.pers_len[(size_t)bh * S + s] : 0;
-            if (len < 0 || len > 64 || (len & 7)) {
+            if (len < 0 || len > 64) {
                 set_status(a.status, PBSA_ERR_DEVICE_CHECK);
                 len = 0;
             }
-            const int ng = len >> 3, oc = ng > 0 ? 1 : 0;
+            const int ng = (len + 7) >> 3, oc = ng > 0 ? 1 : 0;
             int inc_g = ng, inc_o = oc;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
@@ -310,7 +265,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
             if (ng > 0) {
                 seg_slot[rank] = s;
                 for (int i = 0; i < ng; ++i) {
-                    grp_row[gstart + i] = ((bh * S) + s) * 64 + 8 * i;
+                    grp_row[gstart + i] = (((bh * S) + s) * 64 + 8 * i) | (min(8, len - 8 * i) & 7);
                     grp_seg[gstart + i] = rank;
                 }
             }
@@ -322,15 +277,22 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
             misc[M_OCC] = occ;
         }
         __syncwarp();
-        // per 16-group tile: bit g set when group g is the last group of its slot
+        // per 16-group tile: bit g set when group g is the last group of its slot, and the
+        // valid key columns (8 per group, fewer in a slot's partial last group, none past G)
         for (int t = lane; t * 16 < run; t += 32) {
             uint32_t ends = 0;
+            uint32_t mw[4] = {0u, 0u, 0u, 0u};
             for (int gq = 0; gq < 16; ++gq) {
                 const int gi = 16 * t + gq;
                 if (gi < run && (gi + 1 == run || grp_seg[gi + 1] != grp_seg[gi])) ends |= 1u << gq;
+                if (gi < run) {
+                    const int nv = grp_row[gi] & 7;
+                    mw[gq >> 2] |= (nv ? ((1u << nv) - 1u) : 0xffu) << (8 * (gq & 3));
+                }
             }
             tile_end[t] = ends;
             tile_seg[t] = grp_seg[16 * t];
+            tile_mask[t] = make_uint4(mw[0], mw[1], mw[2], mw[3]);
         }
     }
     if ((warp == 1 || warp == 2) && lane == 0) {
@@ -556,30 +518,34 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
             };
             load_s();
             const bool persistent = k < n_pt;
-            int lj = 0;
-            bool masked;
-            uint64_t mk0 = ~0ull, mk1 = ~0ull;
-            if (persistent) {
-                const int nvc = min(128, 8 * (G - 16 * k));
-                masked = nvc < 128;
-                if (masked) {
-                    mk0 = prefix_mask(min(nvc, 64));
-                    mk1 = prefix_mask(max(nvc - 64, 0));
+            const int lj = persistent ? 0 : k - n_pt;
+            // valid-column masks of the tile (64 bits per half); recomputed where they are
+            // applied so that only the `masked` flag stays live across the exponentials
+            auto tile_masks = [&](uint64_t& m0, uint64_t& m1) {
+                if (persistent) {
+                    const uint4 tm = tile_mask[k];
+                    m0 = (static_cast<uint64_t>(tm.y) << 32) | tm.x;
+                    m1 = (static_cast<uint64_t>(tm.w) << 32) | tm.z;
+                } else {
+                    const int u0 = 2 * lj;
+                    const bool has1 = u0 + 1 < U;
+                    const int L0 = ublk[u0], L1 = has1 ? ublk[u0 + 1] : L0;
+                    const bool sel0 = (ubits[u0] >> hq) & 1;
+                    const bool sel1 = has1 && ((ubits[u0 + 1] >> hq) & 1);
+                    const int i0 = L0 % g.nbf, i1 = L1 % g.nbf;
+                    m0 = block_mask(sel0, min(8, g.fh - 8 * (i0 / g.nbx)), min(8, g.fw - 8 * (i0 % g.nbx)));
+                    m1 = block_mask(sel1, min(8, g.fh - 8 * (i1 / g.nbx)), min(8, g.fw - 8 * (i1 % g.nbx)));
                 }
-            } else {
-                lj = k - n_pt;
-                const int u0 = 2 * lj;
-                const bool has1 = u0 + 1 < U;
-                const int L0 = ublk[u0], L1 = has1 ? ublk[u0 + 1] : L0;
-                const bool sel0 = (ubits[u0] >> hq) & 1;
-                const bool sel1 = has1 && ((ubits[u0 + 1] >> hq) & 1);
-                const int i0 = L0 % g.nbf, i1 = L1 % g.nbf;
-                mk0 = block_mask(sel0, min(8, g.fh - 8 * (i0 / g.nbx)), min(8, g.fw - 8 * (i0 % g.nbx)));
-                mk1 = block_mask(sel1, min(8, g.fh - 8 * (i1 / g.nbx)), min(8, g.fw - 8 * (i1 % g.nbx)));
-                masked = true;
+            };
+            bool masked;
+            {
+                uint64_t m0, m1;
+                tile_masks(m0, m1);
+                masked = (m0 & m1) != ~0ull;
             }
-            masked = masked && (mk0 != ~0ull || mk1 != ~0ull);
             auto apply_mask = [&]() {
+                uint64_t mk0, mk1;
+                tile_masks(mk0, mk1);
 #pragma unroll
                 for (int c = 0; c < 64; ++c) {
                     if (!((mk0 >> c) & 1ull)) x[c] = -CUDART_INF_F;
@@ -595,7 +561,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
             // first half.
             float gs[16];
             const float mu0 = (m == -CUDART_INF_F) ? 0.f : m;
-            const float mt = masked ? exp_half0_max<0>(x, sl2, mu0, gs) : exp_half0_max<kEmuPairs>(x, sl2, mu0, gs);
+            const float mt = exp_half0_max(x, sl2, mu0, gs);
             const float m_new = fmaxf(m, mt * sl2);
             const bool need = m_new > m + 8.0f;
             if (__any_sync(0xffffffffu, need)) {
@@ -622,7 +588,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                 }
                 load_s();
                 if (masked) apply_mask();
-                exp_half<0, 0>(x, sl2, (m == -CUDART_INF_F) ? 0.f : m, gs);
+                exp_half<0>(x, sl2, (m == -CUDART_INF_F) ? 0.f : m, gs);
             }
             const float mu = (m == -CUDART_INF_F) ? 0.f : m;
             // each half's P (bf16) goes over the first 64 columns of S as soon as it is done, so
@@ -632,8 +598,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
 #pragma unroll
                 for (int e = 0; e < 32; ++e) v0[e] = pack_bf16x2(x[2 * e], x[2 * e + 1]);
                 tmem_st32(s_addr, v0);
-                if (masked) exp_half<0, 1>(x, sl2, mu, gs);
-                else exp_half<kEmuPairs, 1>(x, sl2, mu, gs);
+                exp_half<1>(x, sl2, mu, gs);
 #pragma unroll
                 for (int e = 0; e < 32; ++e) v1[e] = pack_bf16x2(x[64 + 2 * e], x[64 + 2 * e + 1]);
                 tmem_st32(s_addr + 32, v1);

@@ -302,10 +302,11 @@ __device__ __forceinline__ void tmem_st_wait() {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
-// Loads 16 compacted 8-row groups (rows grp_row[first..first+15] of a [rows, D] slot store,
-// the last group repeated past G) into a K-major SW128 tile: group c of 64-channel half hh
-// lands at dst + hh * half_bytes + 1024 c.  Eight groups that are 64 contiguous rows (a full
-// slot, or full slots back to back) go as one 64-row box instead of eight 8-row boxes.
+// Loads 16 compacted 8-row groups (first rows grp_row[first..first+15] & ~7 of a [rows, D]
+// slot store; the low 3 bits of an entry carry the group's valid-row count and are ignored
+// here; the last group is repeated past G) into a K-major SW128 tile: group c of 64-channel
+// half hh lands at dst + hh * half_bytes + 1024 c.  Eight groups that are 64 contiguous rows
+// (a full slot, or full slots back to back) go as one 64-row box instead of eight 8-row boxes.
 template <int NH>
 __device__ __forceinline__ void tma_load_groups16(uint8_t* dst, uint32_t half_bytes, const CUtensorMap* m8,
                                                   const CUtensorMap* m64, const int32_t* grp_row,
@@ -313,8 +314,8 @@ __device__ __forceinline__ void tma_load_groups16(uint8_t* dst, uint32_t half_by
     int c = 0;
     while (c < 16) {
         const int gi = first + c;
-        const int row = grp_row[gi < G ? gi : G - 1];
-        if ((c & 7) == 0 && gi + 7 < G && grp_row[gi + 7] == row + 56) {
+        const int row = grp_row[gi < G ? gi : G - 1] & ~7;
+        if ((c & 7) == 0 && gi + 7 < G && (grp_row[gi + 7] & ~7) == row + 56) {
 #pragma unroll
             for (int hh = 0; hh < NH; ++hh) tma_load_2d(dst + hh * half_bytes + c * 1024, m64, bar, hh * 64, row);
             c += 8;

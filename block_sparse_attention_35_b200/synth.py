@@ -18,7 +18,7 @@ import math
 import torch
 
 __all__ = ["Workload", "WORKLOADS", "block_extents", "decode_inputs", "rollout_chunk",
-           "training_inputs", "slot_count"]
+           "rollout_chunk_hot", "training_inputs", "slot_count"]
 
 
 @dataclasses.dataclass(frozen=True)
@@ -200,6 +200,34 @@ def rollout_chunk(wl: Workload, step: int):
     k = _normal(gen, shape, wl.value_std).to(bf)
     v = _normal(gen, shape, wl.value_std).to(bf)
     return q, k, v
+
+
+def rollout_chunk_hot(wl: Workload, step: int, q_bias: float = 4.0, hot_bias: float = 4.0,
+                      hot_fraction: float = 0.1):
+    """Like rollout_chunk, but every query token carries q_bias * u and a seeded
+    hot_fraction of the chunk's key blocks carry hot_bias * u on every token, u being one
+    seeded unit vector per (batch, head) shared by all chunks: a stream in which some new
+    blocks keep drawing most of the queries' attention."""
+    q, k, v = rollout_chunk(wl, step)
+    gu = torch.Generator().manual_seed(wl.seed * 7919 + 1)
+    u = torch.stack([torch.stack([_unit(gu, wl.D) for _ in range(wl.H)]) for _ in range(wl.B)])
+    gen = torch.Generator().manual_seed(wl.seed * 1000033 + step)
+    qf = q.float() + q_bias * u[:, None]
+    kf = k.float()
+    ext = block_extents(wl.frame_h, wl.frame_w, wl.block[1], wl.block[2])
+    nbx = -(-wl.frame_w // wl.block[2])
+    nblk = wl.q_frames * len(ext)
+    nhot = max(1, int(round(hot_fraction * nblk)))
+    kv = kf.view(wl.B, wl.q_frames, wl.frame_h, wl.frame_w, wl.H, wl.D)
+    bh, bw = wl.block[1], wl.block[2]
+    for b in range(wl.B):
+        for h in range(wl.H):
+            for j in torch.randperm(nblk, generator=gen)[:nhot].tolist():
+                f, i = divmod(j, len(ext))
+                by, bx = divmod(i, nbx)
+                kv[b, f, by * bh:by * bh + bh, bx * bw:bx * bw + bw, h, :] += hot_bias * u[b, h]
+    bf = torch.bfloat16
+    return qf.to(bf), kf.to(bf), v
 
 
 def training_inputs(wl: Workload, frames: int | None = None):

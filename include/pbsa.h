@@ -36,9 +36,13 @@
  *                            ring slot (ring_head + p) % W.
  *      key_persistent / value_persistent [B, H, S, 64, D]   bf16: S slots of one block
  *                            each, the block's tokens in raster order in rows
- *                            0 .. pers_len-1 (rows past pers_len are ignored).
- *      pers_len [B, H, S] int32 (0 = empty slot, else the block's token count, a
- *                            multiple of 8 for 8x8 blocks cut by the frame edge).
+ *                            0 .. pers_len-1.  Rows past pers_len never reach an output
+ *                            but must hold finite values (pbsa_cache_update leaves them
+ *                            zero): the kernels stream slots in 8-row groups and multiply
+ *                            the masked rows by an exact zero.
+ *      pers_len [B, H, S] int32 (0 = empty slot, else the block's token count, 1..64:
+ *                            64 for an interior 8x8 block, hv * wv for a block cut by
+ *                            the frame edge, e.g. 6 x 2 = 12 on a 30 x 50 grid).
  *  - Blocks: 1 x 8 x 8 tokens; a frame has NB_f = ceil(frame_h/8) * ceil(frame_w/8)
  *    blocks numbered by * ceil(frame_w/8) + bx; edge blocks are clipped to the frame.
  *    Local block ids are LOGICAL: window frame p, block i -> p * NB_f + i.  Query block
