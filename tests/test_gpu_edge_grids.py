@@ -4,8 +4,6 @@ Persistent slots then carry lengths such as 12, 15 or 20, both in the synthetic 
 cache and after a merge admits edge blocks.  Each case runs, through the C ABI, select ->
 forward with block mass -> slide + merge -> forward on the merged cache -> backward, and
 compares every step with the fp64 oracle on the same inputs."""
-import dataclasses
-
 import numpy as np
 import pytest
 import torch
@@ -186,5 +184,10 @@ def test_slot_rows_past_length_do_not_leak(cuda_dev):
         assert int(buf.status.item()) == 0
         outs.append((buf.out.clone(), buf.lse.clone(), buf.mass_pers.clone(), g["dq"].clone(),
                      g["dkl"].clone()))
-    for a, b in zip(*outs):
-        assert torch.equal(a, b)
+    # outputs, lse and gradients are deterministic; the masses are summed across CTAs with
+    # atomics in any order, so they agree to rounding
+    for i, (a, b) in enumerate(zip(*outs)):
+        if i == 2:
+            assert torch.allclose(a, b, rtol=1e-6, atol=0)
+        else:
+            assert torch.equal(a, b)
