@@ -44,42 +44,48 @@ __all__ = ["frame_blocks", "topk_count", "pool_blocks", "block_scores", "select_
 
 
 # ---------------------------------------------------------------------------------------
-# Geometry (project page, usage snippet: sparse_kv_block_size=[1, 8, 8])
+# Geometry (project page, usage snippet: sparse_kv_block_size=[1, 8, 8]; the comparison
+# table's "[3,4,4] block size" rows: blocks of 3 frames x 4 x 4 tokens)
 # ---------------------------------------------------------------------------------------
-def frame_blocks(frame_h: int, frame_w: int, bh: int = 8, bw: int = 8):
-    """Token indices of each 1 x bh x bw block of one frame.
+def frame_blocks(frame_h: int, frame_w: int, bh: int = 8, bw: int = 8, bt: int = 1):
+    """Token indices of each bt x bh x bw block of one group of bt consecutive frames.
 
-    Tokens of a frame are numbered in raster order (n = y * frame_w + x).  Blocks are
-    numbered row of blocks first: id = by * ceil(frame_w / bw) + bx.  Edge blocks are
-    clipped to the frame (reading: ragged blocks hold only their valid tokens).  Inside a
-    block tokens are listed in raster order; this is also the row order of a block copied
-    into a persistent slot.
+    Tokens of a frame are numbered in raster order (n = y * frame_w + x) and the frames of
+    a group follow one another, so token (t, y, x) of the group is t * frame_h * frame_w +
+    y * frame_w + x.  Blocks are numbered row of blocks first: id = by * ceil(frame_w / bw)
+    + bx; every block spans all bt frames of the group.  Edge blocks are clipped to the
+    frame (reading: ragged blocks hold only their valid tokens).  Inside a block tokens are
+    listed frame by frame, each frame in raster order; this is also the row order of a
+    block copied into a persistent slot.  With bt = 1 a group is one frame.
     """
+    tf = frame_h * frame_w
     out = []
     for y0 in range(0, frame_h, bh):
         for x0 in range(0, frame_w, bw):
-            toks = [y * frame_w + x
+            toks = [t * tf + y * frame_w + x
+                    for t in range(bt)
                     for y in range(y0, min(y0 + bh, frame_h))
                     for x in range(x0, min(x0 + bw, frame_w))]
             out.append(np.asarray(toks, dtype=np.int64))
     return out
 
 
-def slot_capacity(bh: int = 8, bw: int = 8) -> int:
-    """Rows of one persistent slot: one full block."""
-    return bh * bw
+def slot_capacity(bh: int = 8, bw: int = 8, bt: int = 1) -> int:
+    """Tokens of one full block, which one persistent slot holds."""
+    return bt * bh * bw
 
 
-def n_slots(persistent_cache_size: int, frame_h: int, frame_w: int, bh=8, bw=8) -> int:
-    """Persistent capacity in blocks (reading: the token budget of whole frames' blocks)."""
-    tf = frame_h * frame_w
-    if persistent_cache_size % tf == 0:
-        return persistent_cache_size // tf * len(frame_blocks(frame_h, frame_w, bh, bw))
-    return -(-persistent_cache_size // (bh * bw))
+def n_slots(persistent_cache_size: int, frame_h: int, frame_w: int, bh=8, bw=8, bt=1) -> int:
+    """Persistent capacity in blocks (reading: the blocks of the whole frame groups the token
+    budget holds; otherwise the budget in full blocks, rounded up)."""
+    tg = bt * frame_h * frame_w
+    if persistent_cache_size % tg == 0:
+        return persistent_cache_size // tg * len(frame_blocks(frame_h, frame_w, bh, bw, bt))
+    return -(-persistent_cache_size // (bt * bh * bw))
 
 
 def cache_geometry(kv_cache_mode: str, total_cache_size: int, local_cache_size: int,
-                   persistent_cache_size: int, frame_h: int, frame_w: int, bh=8, bw=8):
+                   persistent_cache_size: int, frame_h: int, frame_w: int, bh=8, bw=8, bt=1):
     """(window frames W, persistent slots S, every window block attended?) of a cache mode.
 
     kv_cache_mode="sparse_forcing" (project page, constructor default): a window of
@@ -92,7 +98,7 @@ def cache_geometry(kv_cache_mode: str, total_cache_size: int, local_cache_size: 
         return total_cache_size // tf, 0, True
     if kv_cache_mode != "sparse_forcing":
         raise ValueError(kv_cache_mode)
-    return local_cache_size // tf, n_slots(persistent_cache_size, frame_h, frame_w, bh, bw), False
+    return local_cache_size // tf, n_slots(persistent_cache_size, frame_h, frame_w, bh, bw, bt), False
 
 
 # ---------------------------------------------------------------------------------------
@@ -140,15 +146,16 @@ def select_topk(scores_row: np.ndarray, k: int) -> np.ndarray:
 
 
 def select_blocks(q: np.ndarray, k_win: np.ndarray, frame_h: int, frame_w: int,
-                  ratio: float, use_sparse: bool = True, bh: int = 8, bw: int = 8):
+                  ratio: float, use_sparse: bool = True, bh: int = 8, bw: int = 8, bt: int = 1):
     """Top-k local blocks for every query block.
 
     q:     [B, Fq * T_f, H, D] query chunk.
     k_win: [B, Fw * T_f, H, D] local window, frames oldest first (logical order).
+    Fq and Fw are multiples of bt; block id = frame group * NB + block in group.
     Returns idx [B, H, QB, k] (ascending ids), scores [B, H, QB, N_L].
     """
-    blocks = frame_blocks(frame_h, frame_w, bh, bw)
-    tf = frame_h * frame_w
+    blocks = frame_blocks(frame_h, frame_w, bh, bw, bt)
+    tf = bt * frame_h * frame_w      # tokens of one frame group
     B, nq, H, D = q.shape
     fq, fw = nq // tf, k_win.shape[1] // tf
     n_local = fw * len(blocks)
@@ -217,7 +224,7 @@ def _local_keys(k_win, v_win, b, h, ids, blocks, tf):
 
 
 def attn_fwd(q, k_pers, v_pers, pers_len, k_win, v_win, idx, frame_h, frame_w,
-             bh=8, bw=8, heads=None, qblocks=None):
+             bh=8, bw=8, heads=None, qblocks=None, bt=1):
     """PBSA forward.
 
     q [B, Nq, H, D]; k_pers/v_pers [B, H, S, 64, D] with pers_len [B, H, S];
@@ -228,10 +235,10 @@ def attn_fwd(q, k_pers, v_pers, pers_len, k_win, v_win, idx, frame_h, frame_w,
     Returns O [B, Nq, H, D], lse [B, H, Nq], mass_pers [B, H, S], mass_local [B, H, N_L]
     where mass is the probability summed over the query rows of this chunk, per block.
     `heads` (list of (b, h)) and `qblocks` (list of query block ids) restrict the work to
-    a sample; rows outside it are left NaN in O and lse.
+    a sample; rows outside it are left NaN in O and lse.  Blocks are bt x bh x bw.
     """
-    blocks = frame_blocks(frame_h, frame_w, bh, bw)
-    tf = frame_h * frame_w
+    blocks = frame_blocks(frame_h, frame_w, bh, bw, bt)
+    tf = bt * frame_h * frame_w      # tokens of one frame group
     nbf = len(blocks)
     B, nq, H, D = q.shape
     S = pers_len.shape[2]
@@ -264,7 +271,7 @@ def attn_fwd(q, k_pers, v_pers, pers_len, k_win, v_win, idx, frame_h, frame_w,
 # algorithm fragment: the t=0 pass updates P and L)
 # ---------------------------------------------------------------------------------------
 def cache_update(k_pers, v_pers, pers_len, pers_score, pers_src, k_win, v_win, mass_local,
-                 n_evict_frames, first_frame_global, frame_h, frame_w, bh=8, bw=8):
+                 n_evict_frames, first_frame_global, frame_h, frame_w, bh=8, bw=8, bt=1):
     """Slide the window by n_evict_frames and merge the evicted blocks into the
     persistent set by accumulated attention mass.
 
@@ -282,22 +289,26 @@ def cache_update(k_pers, v_pers, pers_len, pers_score, pers_src, k_win, v_win, m
       the dropped slots in ascending order.  Kept evicted blocks, in id order, fill the
       free slots in that order: the slot receives the block's tokens (raster order inside
       the block), its length, its mass as score and its global id
-      (global frame * NB_f + block in frame) as source.  Dropped slots not refilled end
-      empty (length 0, score 0, source -1).
+      (global frame group * NB + block in group, the group of global frames
+      bt*g .. bt*g + bt - 1 being number g) as source.  Dropped slots not refilled end
+      empty (length 0, score 0, source -1).  n_evict_frames and first_frame_global are
+      multiples of bt.
 
     Returns dict(k_pers, v_pers, pers_len, pers_score, pers_src, updates) where updates
     [b][h] is the list of (slot, logical block id) admissions in admission order.
     """
-    blocks = frame_blocks(frame_h, frame_w, bh, bw)
+    blocks = frame_blocks(frame_h, frame_w, bh, bw, bt)
     nbf = len(blocks)
-    tf = frame_h * frame_w
+    tf = bt * frame_h * frame_w      # tokens of one frame group
+    if n_evict_frames % bt or first_frame_global % bt:
+        raise ValueError("frame counts must be multiples of the block's frame count")
     kp = np.array(k_pers, dtype=np.float64)
     vp = np.array(v_pers, dtype=np.float64)
     plen = np.array(pers_len, dtype=np.int64)
     pscore = np.array(pers_score, dtype=np.float64)
     psrc = np.array(pers_src, dtype=np.int64)
     B, H, S = plen.shape
-    n_ev = n_evict_frames * nbf
+    n_ev = n_evict_frames // bt * nbf
     updates = [[None] * H for _ in range(B)]
     for b in range(B):
         for h in range(H):
@@ -326,7 +337,7 @@ def cache_update(k_pers, v_pers, pers_len, pers_score, pers_src, k_win, v_win, m
                 vp[b, h, s, :n] = np.asarray(v_win[b, toks, h, :], np.float64)
                 plen[b, h, s] = n
                 pscore[b, h, s] = float(mass_local[b, h, j])
-                psrc[b, h, s] = (first_frame_global + f) * nbf + i
+                psrc[b, h, s] = (first_frame_global // bt + f) * nbf + i
                 ups.append((s, j))
             updates[b][h] = ups
     return dict(k_pers=kp, v_pers=vp, pers_len=plen, pers_score=pscore, pers_src=psrc,
@@ -338,7 +349,7 @@ def cache_update(k_pers, v_pers, pers_len, pers_score, pers_src, k_win, v_win, m
 # fixed; gradients flow through the attention only.
 # ---------------------------------------------------------------------------------------
 def attn_bwd(q, k_pers, v_pers, pers_len, k_win, v_win, idx, dO, frame_h, frame_w,
-             bh=8, bw=8, qblocks=None):
+             bh=8, bw=8, qblocks=None, bt=1):
     """Gradients of L = sum(O * dO) for the PBSA forward with the selection idx fixed.
 
     For each query block: P = softmax(q k^T / sqrt(D)) over its key set,
@@ -348,8 +359,8 @@ def attn_bwd(q, k_pers, v_pers, pers_len, k_win, v_win, idx, dO, frame_h, frame_
     length), dK_win/dV_win [B, N_L_tokens, H, D].  `qblocks` restricts the work to the
     contributions of those query blocks (a sample; the other rows of dQ stay zero).
     """
-    blocks = frame_blocks(frame_h, frame_w, bh, bw)
-    tf = frame_h * frame_w
+    blocks = frame_blocks(frame_h, frame_w, bh, bw, bt)
+    tf = bt * frame_h * frame_w      # tokens of one frame group
     nbf = len(blocks)
     B, nq, H, D = q.shape
     S = pers_len.shape[2]
@@ -431,15 +442,15 @@ class DecodeState:
 
     @classmethod
     def empty(cls, B, H, D, S, frame_h, frame_w, bh=8, bw=8):
-        """A rollout's start: empty window, empty persistent cache."""
+        """A rollout's start: empty window, empty persistent cache (64-row slots)."""
         return cls(np.zeros((B, 0, H, D)), np.zeros((B, 0, H, D)), np.zeros((B, H, 0)),
-                   np.zeros((B, H, S, bh * bw, D)), np.zeros((B, H, S, bh * bw, D)),
+                   np.zeros((B, H, S, 64, D)), np.zeros((B, H, S, 64, D)),
                    np.zeros((B, H, S), np.int64), np.zeros((B, H, S)),
                    np.full((B, H, S), -1, np.int64))
 
 
 def decode_step(state: DecodeState, q, k_chunk, v_chunk, ratio, window_frames, frame_h,
-                frame_w, use_sparse=True, idx=None, bh=8, bw=8):
+                frame_w, use_sparse=True, idx=None, bh=8, bw=8, bt=1):
     """One chunk's cache pass, in the order of the algorithm fragment:
 
       1. the chunk's frames join the window (reading: before its attention, so the window
@@ -457,8 +468,7 @@ def decode_step(state: DecodeState, q, k_chunk, v_chunk, ratio, window_frames, f
     Returns (new_state, out) with out = dict(idx, scores, O, lse, mass_pers, mass_local,
     n_evict, updates).  The input state is not modified.
     """
-    blocks = frame_blocks(frame_h, frame_w, bh, bw)
-    nbf = len(blocks)
+    nbf = len(frame_blocks(frame_h, frame_w, bh, bw, bt))
     tf = frame_h * frame_w
     chunk_frames = np.asarray(k_chunk).shape[1] // tf
     frames = state.win_k.shape[1] // tf + chunk_frames
@@ -467,12 +477,12 @@ def decode_step(state: DecodeState, q, k_chunk, v_chunk, ratio, window_frames, f
     win_k = np.concatenate([state.win_k, np.asarray(k_chunk, np.float64)], axis=1)
     win_v = np.concatenate([state.win_v, np.asarray(v_chunk, np.float64)], axis=1)
     B, H = state.pers_len.shape[:2]
-    win_mass = np.concatenate([state.win_mass, np.zeros((B, H, chunk_frames * nbf))], axis=2)
+    win_mass = np.concatenate([state.win_mass, np.zeros((B, H, chunk_frames // bt * nbf))], axis=2)
     scores = None
     if idx is None:
-        idx, scores = select_blocks(q, win_k, frame_h, frame_w, ratio, use_sparse, bh, bw)
+        idx, scores = select_blocks(q, win_k, frame_h, frame_w, ratio, use_sparse, bh, bw, bt)
     O, lse, mass_pers, mass_local = attn_fwd(q, state.k_pers, state.v_pers, state.pers_len,
-                                             win_k, win_v, idx, frame_h, frame_w, bh, bw)
+                                             win_k, win_v, idx, frame_h, frame_w, bh, bw, bt=bt)
     win_mass = win_mass + mass_local
     pers_score = state.pers_score + mass_pers
     n_ev = evict_count(frames, chunk_frames, window_frames)
@@ -485,9 +495,9 @@ def decode_step(state: DecodeState, q, k_chunk, v_chunk, ratio, window_frames, f
         return new, out
     r = cache_update(state.k_pers, state.v_pers, state.pers_len, pers_score, state.pers_src,
                      win_k, win_v, win_mass, n_ev, state.first_frame_global, frame_h, frame_w,
-                     bh, bw)
+                     bh, bw, bt)
     out["updates"] = r["updates"]
-    new = DecodeState(win_k[:, n_ev * tf:], win_v[:, n_ev * tf:], win_mass[:, :, n_ev * nbf:],
+    new = DecodeState(win_k[:, n_ev * tf:], win_v[:, n_ev * tf:], win_mass[:, :, n_ev // bt * nbf:],
                       r["k_pers"], r["v_pers"], r["pers_len"], r["pers_score"], r["pers_src"],
                       state.first_frame_global + n_ev)
     return new, out

@@ -573,3 +573,139 @@ def test_decode_step_hand_rollout_fill_admit_and_turnover():
     assert st3.pers_len.tolist() == [[[64, 64]]]
     assert (st3.k_pers[0, 0, 1, :, 0] == 10.0).all() and (st3.k_pers[0, 0, 1, :, 1:] == 0).all()
     assert st3.first_frame_global == 3 and st3.win_k.shape[1] == 128
+
+
+# --------------------------------------------- [3,4,4] blocks (3 frames x 4 x 4 tokens)
+def _block_of(pos, fh, fw, bt, bh, bw):
+    """Block id of a token from its coordinates: position pos in a frame-major sequence ->
+    frame, row, column -> (frame group, block row, block column)."""
+    tf = fh * fw
+    f, n = divmod(pos, tf)
+    y, x = divmod(n, fw)
+    nbx = -(-fw // bw)
+    return (f // bt) * (-(-fh // bh) * nbx) + (y // bh) * nbx + x // bw
+
+
+def test_frame_blocks_344_partition_30x52():
+    blocks = orc.frame_blocks(30, 52, 4, 4, 3)
+    assert len(blocks) == 8 * 13                       # 8 block rows (the last 2 high) x 13
+    sizes = sorted(len(b) for b in blocks)
+    assert sizes == sorted([48] * (7 * 13) + [24] * 13)
+    allt = np.sort(np.concatenate(blocks))
+    assert np.array_equal(allt, np.arange(3 * 1560))   # one group of 3 frames, each token once
+    for i, b in enumerate(blocks):
+        assert all(_block_of(p, 30, 52, 3, 4, 4) == i for p in b)
+    # block 0: frames 0-2, rows 0-3, columns 0-3, frame by frame in raster order
+    want = [t * 1560 + y * 52 + x for t in range(3) for y in range(4) for x in range(4)]
+    assert blocks[0].tolist() == want
+    assert orc.n_slots(9360, 30, 52, 4, 4, 3) == 2 * 104
+    assert orc.n_slots(100, 8, 8, 4, 4, 3) == 3       # ceil(100 / 48)
+    assert orc.slot_capacity(4, 4, 3) == 48
+
+
+def test_pool_344_matches_3d_slicing():
+    rng = np.random.default_rng(8)
+    fh, fw, D, G = 10, 8, 3, 2                          # 2 groups of 3 frames
+    x = rng.standard_normal((G * 3 * fh * fw, D))
+    got = orc.pool_blocks(x.reshape(G, 3 * fh * fw, D), orc.frame_blocks(fh, fw, 4, 4, 3))
+    grid = x.reshape(G, 3, fh, fw, D)
+    want = [grid[g, :, y0:y0 + 4, x0:x0 + 4].mean(axis=(0, 1, 2))
+            for g in range(G) for y0 in range(0, fh, 4) for x0 in range(0, fw, 4)]
+    assert np.allclose(got, np.stack(want), rtol=0, atol=1e-14)
+
+
+def _tiny344(seed, B=1, H=2, D=8, fh=6, fw=8, q_groups=1, w_groups=2, S=4, filled=(0, 1, 3)):
+    rng = np.random.default_rng(seed)
+    tg = 3 * fh * fw
+    t = dict(q=rng.standard_normal((B, q_groups * tg, H, D)) * 0.7,
+             kw=rng.standard_normal((B, w_groups * tg, H, D)) * 0.7,
+             vw=rng.standard_normal((B, w_groups * tg, H, D)),
+             kp=np.zeros((B, H, S, 64, D)), vp=np.zeros((B, H, S, 64, D)),
+             plen=np.zeros((B, H, S), np.int64), fh=fh, fw=fw)
+    sizes = [len(b) for b in orc.frame_blocks(fh, fw, 4, 4, 3)]     # 48 and 24 at 6x8
+    for b in range(B):
+        for h in range(H):
+            for n, s in enumerate(filled):
+                L = sizes[(n + h) % len(sizes)]
+                t["plen"][b, h, s] = L
+                t["kp"][b, h, s, :L] = rng.standard_normal((L, D)) * 0.7
+                t["vp"][b, h, s, :L] = rng.standard_normal((L, D))
+    return t
+
+
+def _masked_dense_344(t, idx, b, h, requires_grad=False):
+    """Keys = every persistent row then every window token; a window token is visible to a
+    query token iff the key's block (from its coordinates) is in the query's block list."""
+    fh, fw = t["fh"], t["fw"]
+    nq, nw = t["q"].shape[1], t["kw"].shape[1]
+    T = lambda a: torch.tensor(a, requires_grad=requires_grad)
+    q, kw, vw, kp, vp = T(t["q"][b, :, h]), T(t["kw"][b, :, h]), T(t["vw"][b, :, h]), \
+        T(t["kp"][b, h]), T(t["vp"][b, h])
+    rows = [(s, r) for s in range(kp.shape[0]) for r in range(int(t["plen"][b, h, s]))]
+    keys = torch.cat([torch.stack([kp[s, r] for s, r in rows]), kw])
+    vals = torch.cat([torch.stack([vp[s, r] for s, r in rows]), vw])
+    wb = np.array([_block_of(p, fh, fw, 3, 4, 4) for p in range(nw)])
+    mask = np.zeros((nq, len(keys)), dtype=bool)
+    mask[:, :len(rows)] = True
+    for i in range(nq):
+        mask[i, len(rows):] = np.isin(wb, idx[b, h, _block_of(i, fh, fw, 3, 4, 4)])
+    z = (q @ keys.T / math.sqrt(q.shape[1])).masked_fill(~torch.tensor(mask), -math.inf)
+    p = torch.softmax(z, dim=1)
+    return dict(o=p @ vals, lse=torch.logsumexp(z, 1), p=p, npers=len(rows), wb=wb, rows=rows,
+                leaves=(q, kw, vw, kp, vp))
+
+
+@pytest.mark.parametrize("ratio", [0.25, 0.5])
+def test_fwd_344_equals_masked_dense(ratio):
+    t = _tiny344(seed=21)
+    idx, _ = orc.select_blocks(t["q"], t["kw"], t["fh"], t["fw"], ratio, bh=4, bw=4, bt=3)
+    assert idx.shape[2] == 4 and idx.shape[-1] == orc.topk_count(ratio, 2 * 4)
+    O, lse, mp, ml = orc.attn_fwd(t["q"], t["kp"], t["vp"], t["plen"], t["kw"], t["vw"], idx,
+                                  t["fh"], t["fw"], 4, 4, bt=3)
+    for h in range(t["q"].shape[2]):
+        r = _masked_dense_344(t, idx, 0, h)
+        assert np.allclose(O[0, :, h], r["o"].numpy(), rtol=0, atol=1e-12)
+        assert np.allclose(lse[0, h], r["lse"].numpy(), rtol=0, atol=1e-12)
+        col = r["p"].numpy().sum(axis=0)
+        own = np.array([s for s, _ in r["rows"]])
+        assert np.allclose(mp[0, h], np.bincount(own, col[:r["npers"]], t["plen"].shape[2]), atol=1e-12)
+        assert np.allclose(ml[0, h], np.bincount(r["wb"], col[r["npers"]:], 8), atol=1e-12)
+
+
+def test_bwd_344_matches_torch_autograd_masked_dense():
+    t = _tiny344(seed=22, H=1)
+    idx, _ = orc.select_blocks(t["q"], t["kw"], t["fh"], t["fw"], 0.5, bh=4, bw=4, bt=3)
+    dO = np.random.default_rng(9).standard_normal(t["q"].shape)
+    dQ, dKp, dVp, dKw, dVw = orc.attn_bwd(t["q"], t["kp"], t["vp"], t["plen"], t["kw"], t["vw"],
+                                           idx, dO, t["fh"], t["fw"], 4, 4, bt=3)
+    r = _masked_dense_344(t, idx, 0, 0, requires_grad=True)
+    (r["o"] * torch.tensor(dO[0, :, 0])).sum().backward()
+    q, kw, vw, kp, vp = r["leaves"]
+    for got, want in [(q, dQ[0, :, 0]), (kw, dKw[0, :, 0]), (vw, dVw[0, :, 0]), (kp, dKp[0, 0]),
+                      (vp, dVp[0, 0])]:
+        assert np.allclose(got.grad.numpy(), want, rtol=0, atol=1e-12)
+
+
+def test_merge_344_hand_example():
+    # frames of 4x8 tokens: a group of 3 frames has two 3x4x4 blocks of 48 tokens.  Window of
+    # 2 groups (6 frames), its oldest frame being global frame 6 (group 2).  Slots: 0 holds a
+    # block with score 5, slot 1 is empty.  Evicting one group (3 frames) with masses 3 and
+    # 0.5: candidates 5, 3, 0.5 -> block 0 enters slot 1 with source 2 * 2 + 0 = 4.
+    fh, fw, D = 4, 8, 2
+    tg = 3 * fh * fw
+    kp = np.zeros((1, 1, 2, 64, D))
+    kp[0, 0, 0, :48] = 1.0
+    plen = np.array([[[48, 0]]])
+    kw = np.arange(2 * tg * D, dtype=np.float64).reshape(1, 2 * tg, 1, D)
+    ml = np.array([[[3.0, 0.5, 0.0, 0.0]]])
+    r = orc.cache_update(kp, kp, plen, np.array([[[5.0, 0.0]]]), np.array([[[77, -1]]]), kw, -kw,
+                         ml, 3, 6, fh, fw, 4, 4, bt=3)
+    assert r["updates"][0][0] == [(1, 0)]
+    assert r["pers_len"].tolist() == [[[48, 48]]]
+    assert r["pers_src"].tolist() == [[[77, 4]]]
+    toks = [t * 32 + y * 8 + x for t in range(3) for y in range(4) for x in range(4)]
+    assert np.array_equal(r["k_pers"][0, 0, 1, :48], kw[0, toks, 0])
+    assert np.all(r["k_pers"][0, 0, 1, 48:] == 0)
+    with pytest.raises(ValueError):
+        orc.cache_update(kp, kp, plen, np.zeros((1, 1, 2)), np.zeros((1, 1, 2), int), kw, kw, ml,
+                         2, 6, fh, fw, 4, 4, bt=3)
