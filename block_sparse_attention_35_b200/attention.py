@@ -36,9 +36,12 @@ class SparseForcingAttention:
         P.pbsa_validate_config(self.cfg)
         self.B, self.H, self.D = B, H, D
         self.tf = frame_h * frame_w
-        self.nbf = P.pbsa_blocks_per_frame(self.cfg)
+        self.bt = int(sparse_kv_block_size[0])      # frames per block (a frame group)
+        self.nbf = P.pbsa_blocks_per_frame(self.cfg)  # blocks per frame group
         self.W = P.pbsa_window_frames(self.cfg)
         self.S = P.pbsa_num_slots(self.cfg)
+        if chunk_frames % self.bt:
+            raise ValueError("chunk_frames must be a multiple of the block's frame count")
         self.chunk_frames = chunk_frames
         self.kmax = P.pbsa_topk_count(self.cfg, self.W)
         self.device = torch.device(device)
@@ -54,18 +57,18 @@ class SparseForcingAttention:
         self.pers_len = torch.zeros(B, H, self.S, **i32)
         self.pers_score = torch.zeros(B, H, self.S, **f32)
         self.pers_src = torch.full((B, H, self.S), -1, **i32)
-        self.mass_local = torch.zeros(B, H, self.W * self.nbf, **f32)
+        self.mass_local = torch.zeros(B, H, self.W // self.bt * self.nbf, **f32)
         self.ring_head = 0
         self.local_frames = 0
         self.first_frame_global = 0
         # per-chunk buffers
         qf = chunk_frames
-        qb = qf * self.nbf
+        qb = qf // self.bt * self.nbf
         self.idx = torch.zeros(B, H, qb, self.kmax, **i32)
         self.cnt = torch.zeros(B, H, qb, **i32)
         self.out = torch.empty(B, qf * self.tf, H, D, **bf)
         self.lse = torch.empty(B, H, qf * self.tf, **f32)
-        self.upd = torch.zeros(B, H, self.W * self.nbf, 2, **i32)
+        self.upd = torch.zeros(B, H, self.W // self.bt * self.nbf, 2, **i32)
         self.n_upd = torch.zeros(B, H, **i32)
         self.status = torch.zeros(1, **i32)
         u8 = dict(dtype=torch.uint8, device=dev)

@@ -130,6 +130,16 @@ __device__ __forceinline__ int group_rows(int32_t entry) {
     return nv ? nv : 8;
 }
 
+// Zeroes a CTA's operand tiles (bytes, a multiple of 16) with every thread, then orders
+// those writes before the TMA copies and MMAs that follow.  Blocks of fewer than 64 tokens
+// leave box rows that TMA never writes; they must hold finite values because masked
+// columns multiply them by exact zeros.
+__device__ __forceinline__ void zero_tiles(uint8_t* base, uint32_t bytes) {
+    uint4* z = reinterpret_cast<uint4*>(base);
+    for (uint32_t e = threadIdx.x; e < bytes / 16; e += blockDim.x) z[e] = make_uint4(0, 0, 0, 0);
+    fence_proxy_async_smem();
+}
+
 constexpr int B_COUNT = 12;  // mbarrier slots reserved per CTA
 
 // ===================================================================== dK / dV
@@ -193,9 +203,10 @@ __device__ __forceinline__ void dkdv_body(const BwdKernelArgs& ka, const int cta
 
     const int bh = b * g.H + h;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int qb_total = a.q_frames * g.nbf;
+    const int qb_total = a.q_frames / g.bt * g.nbf;
     const int nq = a.q_frames * g.tf;
-    const int nl = a.local_frames * g.nbf;
+    const int nl = a.local_frames / g.bt * g.nbf;
+    const uint32_t box_bytes = static_cast<uint32_t>(g.brows) * 128u;  // one block, one 64-channel half
     const bool pers_tile = cta_x < ka.n_pt_max;
     const int tile = pers_tile ? cta_x : cta_x - ka.n_pt_max;
 
@@ -219,6 +230,7 @@ __device__ __forceinline__ void dkdv_body(const BwdKernelArgs& ka, const int cta
         misc[1] = 0;
         fence_barrier_init();
     }
+    if (g.brows < 64) zero_tiles(sm + PL.k, PL.lse - PL.k);
     if (warp == kMmaWarp) tmem_alloc(reinterpret_cast<uint32_t*>(misc + 0), 512);
 
     // key set of this CTA
@@ -286,20 +298,20 @@ __device__ __forceinline__ void dkdv_body(const BwdKernelArgs& ka, const int cta
     if (live && warp == kProdWarp) {
         // ---------------------------------------------------------- producer
         if (lane == 0) {
-            mbar_arrive_expect_tx(kv_full, 2 * TILE);
+            mbar_arrive_expect_tx(kv_full, pers_tile ? 2 * TILE : 2 * 2 * NH * box_bytes);
             if (pers_tile) {
                 tma_load_groups16<NH>(sK, kHalf, &a.tm_kp, &a.tm_kp64, grp_row, tile * 16, G, kv_full);
                 tma_load_groups16<NH>(sV, kHalf, &a.tm_vp, &a.tm_vp64, grp_row, tile * 16, G, kv_full);
             } else {
                 for (int kb = 0; kb < 2; ++kb) {
                     const int L = (kb == 1 && L1 >= 0) ? L1 : L0;
-                    const int pos = L / g.nbf, i = L % g.nbf;
-                    const int fr = b * g.W + (a.ring_head + pos) % g.W;
+                    const BlockBox kbb = block_box(g, L % g.nbf);
+                    const int fr = b * g.W + (a.ring_head + (L / g.nbf) * g.bt) % g.W;
                     for (int hh = 0; hh < NH; ++hh) {
                         tma_load_5d(sK + hh * kHalf + kb * (kHalf / 2), &a.tm_kl, kv_full, hh * 64, h,
-                                    8 * (i % g.nbx), 8 * (i / g.nbx), fr);
+                                    kbb.x0, kbb.y0, fr);
                         tma_load_5d(sV + hh * kHalf + kb * (kHalf / 2), &a.tm_vl, kv_full, hh * 64, h,
-                                    8 * (i % g.nbx), 8 * (i / g.nbx), fr);
+                                    kbb.x0, kbb.y0, fr);
                     }
                 }
             }
@@ -316,14 +328,15 @@ __device__ __forceinline__ void dkdv_body(const BwdKernelArgs& ka, const int cta
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
                 const int r = lane + 32 * u;
-                const int hq = r >> 6, qb = 2 * qt + hq, rr = r & 63;
+                const int hq = r >> 6, qb = 2 * qt + hq;
                 l2v[u] = CUDART_INF_F;
                 dlv[u] = 0.f;
                 if (qb < qb_total) {
-                    const int f = qb / g.nbf, i = qb % g.nbf;
-                    const int y = 8 * (i / g.nbx) + (rr >> 3), x = 8 * (i % g.nbx) + (rr & 7);
-                    if (y < g.fh && x < g.fw) {
-                        const size_t t = (size_t)bh * nq + f * g.tf + y * g.fw + x;
+                    const BlockBox qbb = block_box(g, qb % g.nbf);
+                    int tt, y, x;
+                    if (block_row(g, qbb, r & 63, &tt, &y, &x)) {
+                        const size_t t = (size_t)bh * nq + (size_t)((qb / g.nbf) * g.bt + tt) * g.tf +
+                                         (qbb.y0 + y) * g.fw + qbb.x0 + x;
                         l2v[u] = a.lse[t] * kLog2e;
                         dlv[u] = a.delta[t];
                     }
@@ -334,15 +347,16 @@ __device__ __forceinline__ void dkdv_body(const BwdKernelArgs& ka, const int cta
                 if (!w) break;
             }
             if (lane == 0) {
-                mbar_arrive_expect_tx(&qd_full[st], 2 * TILE);
+                mbar_arrive_expect_tx(&qd_full[st], 2 * 2 * NH * box_bytes);
                 for (int hq = 0; hq < 2; ++hq) {
                     const int qb = min(2 * qt + hq, qb_total - 1);
-                    const int f = qb / g.nbf, i = qb % g.nbf;
+                    const BlockBox qbb = block_box(g, qb % g.nbf);
+                    const int f0 = b * a.q_frames + (qb / g.nbf) * g.bt;
                     for (int hh = 0; hh < NH; ++hh) {
                         tma_load_5d(sQ + st * TILE + hh * kHalf + hq * (kHalf / 2), &a.tm_q, &qd_full[st],
-                                    hh * 64, h, 8 * (i % g.nbx), 8 * (i / g.nbx), b * a.q_frames + f);
+                                    hh * 64, h, qbb.x0, qbb.y0, f0);
                         tma_load_5d(sDO + st * TILE + hh * kHalf + hq * (kHalf / 2), &a.tm_do, &qd_full[st],
-                                    hh * 64, h, 8 * (i % g.nbx), 8 * (i / g.nbx), b * a.q_frames + f);
+                                    hh * 64, h, qbb.x0, qbb.y0, f0);
                     }
                 }
             }
@@ -426,8 +440,8 @@ __device__ __forceinline__ void dkdv_body(const BwdKernelArgs& ka, const int cta
             if (L < 0) {
                 key_valid = false;
             } else {
-                const int i = L % g.nbf, rr = r & 63;
-                key_valid = (8 * (i / g.nbx) + (rr >> 3) < g.fh) && (8 * (i % g.nbx) + (rr & 7) < g.fw);
+                int tt, y, x;
+                key_valid = block_row(g, block_box(g, L % g.nbf), r & 63, &tt, &y, &x);
             }
         }
         auto wwait = [&](uint64_t* bar, uint32_t parity) -> bool {
@@ -493,10 +507,12 @@ __device__ __forceinline__ void dkdv_body(const BwdKernelArgs& ka, const int cta
                     dv_row = a.dv_pers + row * D;
                 } else {
                     const int L = kbr ? L1 : L0;
-                    const int pos = L / g.nbf, i = L % g.nbf, rr = r & 63;
-                    const int phys = (a.ring_head + pos) % g.W;
-                    const int y = 8 * (i / g.nbx) + (rr >> 3), x = 8 * (i % g.nbx) + (rr & 7);
-                    const size_t tok = ((size_t)b * g.W + phys) * g.tf + y * g.fw + x;
+                    const BlockBox kbb = block_box(g, L % g.nbf);
+                    int tt, y, x;
+                    block_row(g, kbb, r & 63, &tt, &y, &x);
+                    // ring frame: the group's first frame (groups never wrap the ring) + tt
+                    const int phys = (a.ring_head + (L / g.nbf) * g.bt) % g.W + tt;
+                    const size_t tok = ((size_t)b * g.W + phys) * g.tf + (kbb.y0 + y) * g.fw + kbb.x0 + x;
                     dk_row = a.dk_local + (tok * g.H + h) * D;
                     dv_row = a.dv_local + (tok * g.H + h) * D;
                 }
@@ -538,10 +554,10 @@ __device__ __forceinline__ void dkdv_body(const BwdKernelArgs& ka, const int cta
 
 // ========================================================================== dQ
 struct DqPlan {
-    uint32_t q, dq_o, k, v, grp_row, uni_blk, uni_bits, bars, misc, total;
+    uint32_t q, dq_o, k, v, grp_row, uni_blk, uni_bits, blk_mask, bars, misc, total;
 };
 
-__host__ __device__ inline DqPlan dq_plan(int D, int S, int ucap) {
+__host__ __device__ inline DqPlan dq_plan(int D, int S, int ucap, int nbf) {
     DqPlan p;
     const uint32_t nh = D / 64;
     p.q = 0;
@@ -551,7 +567,8 @@ __host__ __device__ inline DqPlan dq_plan(int D, int S, int ucap) {
     p.grp_row = p.v + kNst * nh * kHalf;
     p.uni_blk = p.grp_row + 4u * 8u * S;
     p.uni_bits = p.uni_blk + 4u * ucap;
-    p.bars = (p.uni_bits + 4u * ucap + 7u) & ~7u;
+    p.blk_mask = (p.uni_bits + 4u * ucap + 7u) & ~7u;  // [nbf] valid rows of each block
+    p.bars = p.blk_mask + 8u * nbf;
     p.misc = p.bars + 8u * 16u;
     p.total = p.misc + 4u * 8u;
     return p;
@@ -571,7 +588,7 @@ __device__ __forceinline__ void dq_body(const BwdKernelArgs& ka, const int tile,
                                              ~static_cast<uintptr_t>(1023));
     const int S = g.S;
     const int ucap = ka.ucap;
-    const DqPlan PL = dq_plan(D, S, ucap);
+    const DqPlan PL = dq_plan(D, S, ucap, g.nbf);
     uint8_t* sQ = sm + PL.q;
     uint8_t* sDO = sm + PL.dq_o;
     uint8_t* sK = sm + PL.k;
@@ -579,6 +596,7 @@ __device__ __forceinline__ void dq_body(const BwdKernelArgs& ka, const int tile,
     int32_t* grp_row = reinterpret_cast<int32_t*>(sm + PL.grp_row);
     int32_t* uni_blk = reinterpret_cast<int32_t*>(sm + PL.uni_blk);
     int32_t* uni_bits = reinterpret_cast<int32_t*>(sm + PL.uni_bits);
+    uint64_t* blk_mask = reinterpret_cast<uint64_t*>(sm + PL.blk_mask);
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + PL.bars);
     int* misc = reinterpret_cast<int*>(sm + PL.misc);
     volatile int* abort_flag = misc + 1;
@@ -592,11 +610,12 @@ __device__ __forceinline__ void dq_body(const BwdKernelArgs& ka, const int tile,
     uint64_t* drain = &bars[10];
 
     const int bh = b * g.H + h;
-    const int qb_total = a.q_frames * g.nbf;
+    const int qb_total = a.q_frames / g.bt * g.nbf;
     const int nq = a.q_frames * g.tf;
     const int qb0 = 2 * tile;
     const int qb1 = (2 * tile + 1 < qb_total) ? 2 * tile + 1 : -1;
-    const int nl = a.local_frames * g.nbf;
+    const int nl = a.local_frames / g.bt * g.nbf;
+    const uint32_t box_bytes = static_cast<uint32_t>(g.brows) * 128u;  // one block, one 64-channel half
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
@@ -613,6 +632,8 @@ __device__ __forceinline__ void dq_body(const BwdKernelArgs& ka, const int tile,
         misc[1] = 0;
         fence_barrier_init();
     }
+    for (int i = threadIdx.x; i < g.nbf; i += blockDim.x) blk_mask[i] = block_rows_mask(g, i);
+    if (g.brows < 64) zero_tiles(sm + PL.q, PL.grp_row - PL.q);
     if (warp == kMmaWarp) tmem_alloc(reinterpret_cast<uint32_t*>(misc + 0), 512);
     if (warp == 0) {
         const int G = build_groups(a.pers_len, bh, S, grp_row, a.status);
@@ -659,15 +680,14 @@ __device__ __forceinline__ void dq_body(const BwdKernelArgs& ka, const int tile,
 
     if (warp == kProdWarp) {
         if (lane == 0) {
-            mbar_arrive_expect_tx(q_full, 2 * TILE);
+            mbar_arrive_expect_tx(q_full, 2 * 2 * NH * box_bytes);
             for (int hb = 0; hb < 2; ++hb) {
                 const int qb = (hb == 1 && qb1 >= 0) ? qb1 : qb0;
-                const int f = qb / g.nbf, i = qb % g.nbf;
+                const BlockBox qbb = block_box(g, qb % g.nbf);
+                const int f0 = b * a.q_frames + (qb / g.nbf) * g.bt;
                 for (int hh = 0; hh < NH; ++hh) {
-                    tma_load_5d(sQ + hh * kHalf + hb * (kHalf / 2), &a.tm_q, q_full, hh * 64, h,
-                                8 * (i % g.nbx), 8 * (i / g.nbx), b * a.q_frames + f);
-                    tma_load_5d(sDO + hh * kHalf + hb * (kHalf / 2), &a.tm_do, q_full, hh * 64, h,
-                                8 * (i % g.nbx), 8 * (i / g.nbx), b * a.q_frames + f);
+                    tma_load_5d(sQ + hh * kHalf + hb * (kHalf / 2), &a.tm_q, q_full, hh * 64, h, qbb.x0, qbb.y0, f0);
+                    tma_load_5d(sDO + hh * kHalf + hb * (kHalf / 2), &a.tm_do, q_full, hh * 64, h, qbb.x0, qbb.y0, f0);
                 }
             }
             int issued = 0;
@@ -676,8 +696,9 @@ __device__ __forceinline__ void dq_body(const BwdKernelArgs& ka, const int tile,
                 if (it >= kNst && !mbar_wait(&kv_empty[st], ((it / kNst) - 1) & 1, abort_flag, a.status)) break;
                 uint8_t* dk = sK + st * TILE;
                 uint8_t* dv = sV + st * TILE;
-                mbar_arrive_expect_tx(&k_full[st], TILE);
-                mbar_arrive_expect_tx(&v_full[st], TILE);
+                const uint32_t tile_bytes = it < n_pt ? TILE : 2 * NH * box_bytes;
+                mbar_arrive_expect_tx(&k_full[st], tile_bytes);
+                mbar_arrive_expect_tx(&v_full[st], tile_bytes);
                 if (it < n_pt) {
                     for (int c = 0; c < 16; ++c) {
                         const int row = grp_row[min(it * 16 + c, G - 1)] & ~7;
@@ -690,13 +711,13 @@ __device__ __forceinline__ void dq_body(const BwdKernelArgs& ka, const int tile,
                     const int j = it - n_pt;
                     for (int hb = 0; hb < 2; ++hb) {
                         const int L = uni_blk[min(2 * j + hb, U - 1)];
-                        const int pos = L / g.nbf, i = L % g.nbf;
-                        const int fr = b * g.W + (a.ring_head + pos) % g.W;
+                        const BlockBox kbb = block_box(g, L % g.nbf);
+                        const int fr = b * g.W + (a.ring_head + (L / g.nbf) * g.bt) % g.W;
                         for (int hh = 0; hh < NH; ++hh) {
                             tma_load_5d(dk + hh * kHalf + hb * (kHalf / 2), &a.tm_kl, &k_full[st], hh * 64, h,
-                                        8 * (i % g.nbx), 8 * (i / g.nbx), fr);
+                                        kbb.x0, kbb.y0, fr);
                             tma_load_5d(dv + hh * kHalf + hb * (kHalf / 2), &a.tm_vl, &v_full[st], hh * 64, h,
-                                        8 * (i % g.nbx), 8 * (i / g.nbx), fr);
+                                        kbb.x0, kbb.y0, fr);
                         }
                     }
                 }
@@ -756,13 +777,13 @@ __device__ __forceinline__ void dq_body(const BwdKernelArgs& ka, const int tile,
         const int r = 32 * wq + lane;
         const int c0 = kCw * cg;              // first key column of this warp
         const int kh = c0 >> 6;               // key block (half of a local key tile) of those columns
-        const int hq = r >> 6, rr = r & 63, dy = rr >> 3, dx = rr & 7;
+        const int hq = r >> 6;
         const int qbr = hq ? qb1 : qb0;
         const int qbv = qbr >= 0 ? qbr : qb0;
-        const int qf = qbv / g.nbf, qi = qbv % g.nbf;
-        const int qy = 8 * (qi / g.nbx) + dy, qx = 8 * (qi % g.nbx) + dx;
-        const bool row_valid = qbr >= 0 && qy < g.fh && qx < g.fw;
-        const size_t tok = (size_t)qf * g.tf + qy * g.fw + qx;
+        const BlockBox qbb = block_box(g, qbv % g.nbf);
+        int qt, qy, qx;
+        const bool row_valid = block_row(g, qbb, r & 63, &qt, &qy, &qx) && qbr >= 0;
+        const size_t tok = (size_t)((qbv / g.nbf) * g.bt + qt) * g.tf + (qbb.y0 + qy) * g.fw + qbb.x0 + qx;
         const float lse2 = row_valid ? a.lse[(size_t)bh * nq + tok] * kLog2e : CUDART_INF_F;
         const float dl = row_valid ? a.delta[(size_t)bh * nq + tok] : 0.f;
         const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
@@ -792,17 +813,8 @@ __device__ __forceinline__ void dq_body(const BwdKernelArgs& ka, const int tile,
                 const bool has = u < U;
                 const int L = uni_blk[has ? u : 0];
                 const bool sel = has && ((uni_bits[has ? u : 0] >> hq) & 1);
-                const int i = L % g.nbf;
-                const int hv = min(8, g.fh - 8 * (i / g.nbx)), wv = min(8, g.fw - 8 * (i % g.nbx));
-                // columns c0.. are in-block positions (c0 & 63) + e = 8 y + x
-                const uint32_t rowbits = wv >= 8 ? 0xffu : ((1u << wv) - 1u);
-                uint32_t m = 0;
-#pragma unroll
-                for (int yy = 0; yy < kCw / 8; ++yy) {
-                    const int y = ((c0 & 63) >> 3) + yy;
-                    if (y < hv) m |= rowbits << (8 * yy);
-                }
-                vmask = sel ? m : 0u;
+                // columns c0.. are the block's box rows (c0 & 63) + e
+                vmask = sel ? static_cast<uint32_t>(blk_mask[L % g.nbf] >> (c0 & 63)) : 0u;
             }
             uint32_t dk[kCw / 2];
 #pragma unroll
@@ -895,9 +907,9 @@ cudaError_t launch_k(K kernel, const A& args, dim3 grid, size_t smem, cudaStream
 }  // namespace
 
 size_t attn_bwd_smem_bytes(const Geo& g, int q_frames, int ucap) {
-    const int n_qt = (q_frames * g.nbf + 1) / 2;
+    const int n_qt = (q_frames / g.bt * g.nbf + 1) / 2;
     const size_t a = dkdv_plan(g.D, g.S, n_qt).total + 1024;
-    const size_t b = dq_plan(g.D, g.S, ucap).total + 1024;
+    const size_t b = dq_plan(g.D, g.S, ucap, g.nbf).total + 1024;
     size_t m = a > b ? a : b;
     return m < 120 * 1024 ? 120 * 1024 : m;
 }
@@ -910,14 +922,14 @@ cudaError_t launch_attn_bwd(const BwdArgs& a, cudaStream_t st) {
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
 
-    const int qb_total = a.q_frames * g.nbf;
+    const int qb_total = a.q_frames / g.bt * g.nbf;
     BwdKernelArgs ka;
     ka.a = a;
     ka.n_pt_max = (g.S * 8 + 15) / 16;
     ka.n_qt = (qb_total + 1) / 2;
     ka.ucap = a.ucap;
     ka.n_dq_x = (qb_total + 1) / 2;
-    ka.n_kd_x = ka.n_pt_max + (a.local_frames * g.nbf + 1) / 2;
+    ka.n_kd_x = ka.n_pt_max + (a.local_frames / g.bt * g.nbf + 1) / 2;
     const size_t smem = attn_bwd_smem_bytes(g, a.q_frames, a.ucap);
     const long long ctas = (long long)(ka.n_dq_x + ka.n_kd_x) * g.H * g.B;
     if (ctas > 0x7fffffffll) return cudaErrorInvalidConfiguration;

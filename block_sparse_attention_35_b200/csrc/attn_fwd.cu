@@ -7,17 +7,18 @@
 // probability summed over the chunk's query rows (the score that ranks blocks when the
 // window slides).
 //
-// One CTA = four 8x8 query blocks of one (batch, head), split into two 128-row query tiles
-// ("sides" A and B, two blocks each, every block a 64-row 5-D TMA box; ragged edge blocks
-// are zero-filled on load and clipped on store).  Key tiles are 128 keys:
+// One CTA = four query blocks of one (batch, head), split into two 128-row query tiles
+// ("sides" A and B, two blocks each; a block is one 5-D TMA box of bt x bh x bw tokens
+// placed in a 64-row half of the tile, rows past bt*bh*bw zero; ragged edge blocks are
+// zero-filled on load and clipped on store).  Key tiles are 128 keys:
 //   * persistent tiles (shared by both sides): the occupied slots' rows compacted into a
 //     stream of 8-row groups (ceil(len / 8) groups per slot; the last group of a slot whose
 //     length is not a multiple of 8 is partly valid and its other rows are masked), 16
 //     groups per tile, loaded as one 64-row TMA box wherever eight groups are contiguous
 //     rows (a full slot);
-//   * local tiles (one side each): the union of that side's two selections, two 8x8 key
-//     blocks per tile; columns the row's query block did not select, or outside the frame,
-//     are masked.  A-tiles and B-tiles alternate in the stream.
+//   * local tiles (one side each): the union of that side's two selections, two key blocks
+//     per tile (one per 64-row half); columns the row's query block did not select, or
+//     outside the block or the frame, are masked.  A-tiles and B-tiles alternate.
 // TMEM (512 columns): S_A | S_B | O_A | O_B.  P (bf16) is written over the first 64 columns
 // of its S and read by a TS MMA; the tensor pipe executes one thread's MMAs in issue order,
 // so S = Q K^T of a side's next tile may be issued right after the O += P V that reads
@@ -58,10 +59,10 @@ constexpr float kLog2e = 1.4426950408889634f;
 
 struct SmemPlan {
     uint32_t q, k, v, grp_row, grp_seg, seg_slot, tile_end, tile_seg, tile_mask, uni_blk, uni_bits,
-        lse_s, bars, misc, total;
+        lse_s, blk_mask, bars, misc, total;
 };
 
-__host__ __device__ inline SmemPlan fwd_plan(int D, int S, int ucap) {
+__host__ __device__ inline SmemPlan fwd_plan(int D, int S, int ucap, int nbf) {
     SmemPlan p;
     const uint32_t nh = D / 64;
     const uint32_t n_pt_max = (8u * S + 15u) / 16u;
@@ -77,7 +78,8 @@ __host__ __device__ inline SmemPlan fwd_plan(int D, int S, int ucap) {
     p.uni_blk = p.tile_mask + 16u * n_pt_max; // [2][ucap]
     p.uni_bits = p.uni_blk + 8u * ucap;      // [2][ucap]
     p.lse_s = p.uni_bits + 8u * ucap;        // [2][128] row log-sum-exp (log2) for the mass
-    p.bars = (p.lse_s + 2u * 128u * 4u + 7u) & ~7u;
+    p.blk_mask = (p.lse_s + 2u * 128u * 4u + 7u) & ~7u;  // [nbf] valid rows of each block
+    p.bars = p.blk_mask + 8u * nbf;
     p.misc = p.bars + 8u * 24u;
     p.total = p.misc + 4u * 16u;
     return p;
@@ -155,14 +157,6 @@ __device__ __forceinline__ void exp_half(float (&x)[128], float sl2, float mu, f
     }
 }
 
-// 64-bit validity mask of one 8x8 key block: rows < hv, columns < wv, all zero if !sel.
-__device__ __forceinline__ uint64_t block_mask(bool sel, int hv, int wv) {
-    if (!sel) return 0ull;
-    const uint64_t rows = hv >= 8 ? ~0ull : ((1ull << (8 * hv)) - 1ull);
-    const uint64_t cols = 0x0101010101010101ull * static_cast<uint64_t>((1u << wv) - 1u);
-    return rows & cols;
-}
-
 // Consumers of stream tile t: bit 0 = side A, bit 1 = side B; *lj = local tile index.
 // Persistent tiles come first (both sides), then the sides' local tiles alternate A, B.
 __device__ __forceinline__ int tile_cons(int t, int n_pt, int nla, int nlb, bool has_b, int* lj) {
@@ -191,7 +185,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                                              ~static_cast<uintptr_t>(1023));
     const int S = g.S;
     const int ucap = a.ucap;
-    const SmemPlan P = fwd_plan(D, S, ucap);
+    const SmemPlan P = fwd_plan(D, S, ucap, g.nbf);
     uint8_t* sQ = sm + P.q;
     uint8_t* sK = sm + P.k;
     uint8_t* sV = sm + P.v;
@@ -204,14 +198,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     int32_t* uni_blk = reinterpret_cast<int32_t*>(sm + P.uni_blk);
     int32_t* uni_bits = reinterpret_cast<int32_t*>(sm + P.uni_bits);
     float* lse_s = reinterpret_cast<float*>(sm + P.lse_s);
+    uint64_t* blk_mask = reinterpret_cast<uint64_t*>(sm + P.blk_mask);
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + P.bars);
     int* misc = reinterpret_cast<int*>(sm + P.misc);
     volatile int* abort_flag = misc + M_ABORT;
 
     const int grp = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int bh = b * g.H + h;
-    const int qb_total = a.q_frames * g.nbf;
-    const int nl = a.local_frames * g.nbf;
+    const int qb_total = a.q_frames / g.bt * g.nbf;
+    const int nl = a.local_frames / g.bt * g.nbf;
+    const int head_g = a.ring_head / g.bt;          // ring frame group of window group 0
+    const uint32_t box_bytes = static_cast<uint32_t>(g.brows) * 128u;  // one block, one 64-channel half
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     // query blocks of the two sides (-1 = none)
     auto qblock = [&](int X, int i) -> int {
@@ -237,6 +234,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         mbar_init(&bars[B_DRAIN], 1);
         misc[M_ABORT] = 0;
         fence_barrier_init();
+    }
+    for (int i = threadIdx.x; i < g.nbf; i += blockDim.x) blk_mask[i] = block_rows_mask(g, i);
+    if (g.brows < 64) {
+        // rows past a block's box are never written by TMA: zero every Q/K/V tile once so
+        // that they hold finite values (masked columns multiply them by exact zeros)
+        uint4* z = reinterpret_cast<uint4*>(sm + P.q);
+        const int n16 = static_cast<int>((P.grp_row - P.q) / 16);
+        for (int e = threadIdx.x; e < n16; e += blockDim.x) z[e] = make_uint4(0, 0, 0, 0);
+        fence_proxy_async_smem();
     }
     if (warp == 10) tmem_alloc(reinterpret_cast<uint32_t*>(misc + M_TMEM), kTmCols);
     if (warp == 0) {
@@ -361,15 +367,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
             tma_prefetch_desc(ml);
             if (isK) {
                 tma_prefetch_desc(&a.tm_q);
-                mbar_arrive_expect_tx(&bars[B_Q], 2 * 2 * NH * (kHalf / 2));
+                mbar_arrive_expect_tx(&bars[B_Q], 2 * 2 * NH * box_bytes);
                 for (int X = 0; X < 2; ++X)
                     for (int hb = 0; hb < 2; ++hb) {
                         int qb = qblock(X, hb);
                         if (qb < 0) qb = qblock(0, 0);  // filler rows, never stored
-                        const int f = qb / g.nbf, i = qb % g.nbf;
+                        const BlockBox qbb = block_box(g, qb % g.nbf);
+                        const int f0 = b * a.q_frames + (qb / g.nbf) * g.bt;
                         for (int hh = 0; hh < NH; ++hh)
                             tma_load_5d(sQ + X * Q_SIDE + hh * kHalf + hb * (kHalf / 2), &a.tm_q, &bars[B_Q],
-                                        hh * 64, h, 8 * (i % g.nbx), 8 * (i / g.nbx), b * a.q_frames + f);
+                                        hh * 64, h, qbb.x0, qbb.y0, f0);
                     }
             }
             int issued = 0;
@@ -377,21 +384,23 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                 const int st = t % kNst;
                 if (t >= kNst && !mbar_wait(&empty[st], ((t / kNst) - 1) & 1, abort_flag, a.status)) break;
                 uint8_t* dst = base + st * KV_BYTES;
-                mbar_arrive_expect_tx(&full[st], KV_BYTES);
                 int lj;
                 const int cons = tile_cons(t, n_pt, nla, nlb, has_b, &lj);
                 if (lj < 0) {
+                    mbar_arrive_expect_tx(&full[st], KV_BYTES);
                     tma_load_groups16<NH>(dst, kHalf, mp, mp64, grp_row, t * 16, G, &full[st]);
                 } else {
+                    mbar_arrive_expect_tx(&full[st], 2 * NH * box_bytes);
                     const int X = cons == 2 ? 1 : 0;
                     const int U = X ? UB : UA;
                     for (int hb = 0; hb < 2; ++hb) {
                         const int L = uni_blk[X * ucap + min(2 * lj + hb, U - 1)];
-                        const int pos = L / g.nbf, i = L % g.nbf;
-                        const int cf = b * g.W + (a.ring_head + pos) % g.W;
+                        const BlockBox kbb = block_box(g, L % g.nbf);
+                        // first ring frame of the block's group (groups never wrap the ring)
+                        const int cf = b * g.W + (a.ring_head + (L / g.nbf) * g.bt) % g.W;
                         for (int hh = 0; hh < NH; ++hh)
                             tma_load_5d(dst + hh * kHalf + hb * (kHalf / 2), ml, &full[st], hh * 64, h,
-                                        8 * (i % g.nbx), 8 * (i / g.nbx), cf);
+                                        kbb.x0, kbb.y0, cf);
                     }
                 }
                 ++issued;
@@ -478,12 +487,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         const int r = threadIdx.x & 127;  // query row of the side's tile = TMEM lane
         const int wq = warp & 3;          // lane quarter
         const int nX = X ? n_side1 : n_side0;
-        const int hq = r >> 6, rr = r & 63, dy = rr >> 3, dx = rr & 7;
+        const int hq = r >> 6;
         const int qbr = qblock(X, hq);
         const int qbv = qbr >= 0 ? qbr : 0;
-        const int qf = qbv / g.nbf, qi = qbv % g.nbf;
-        const int qy = 8 * (qi / g.nbx) + dy, qx = 8 * (qi % g.nbx) + dx;
-        const bool row_valid = qbr >= 0 && qy < g.fh && qx < g.fw;
+        const BlockBox qbb = block_box(g, qbv % g.nbf);
+        int qt, qy, qx;
+        const bool row_valid = block_row(g, qbb, r & 63, &qt, &qy, &qx) && qbr >= 0;
+        // token of this row in the chunk
+        const size_t q_tok = (size_t)((qbv / g.nbf) * g.bt + qt) * g.tf + (qbb.y0 + qy) * g.fw + qbb.x0 + qx;
         const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
         const uint32_t s_col = 128 * X, o_col = 256 + 128 * X;
         const float sl2 = kLog2e / sqrtf(static_cast<float>(D));
@@ -532,9 +543,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                     const int L0 = ublk[u0], L1 = has1 ? ublk[u0 + 1] : L0;
                     const bool sel0 = (ubits[u0] >> hq) & 1;
                     const bool sel1 = has1 && ((ubits[u0 + 1] >> hq) & 1);
-                    const int i0 = L0 % g.nbf, i1 = L1 % g.nbf;
-                    m0 = block_mask(sel0, min(8, g.fh - 8 * (i0 / g.nbx)), min(8, g.fw - 8 * (i0 % g.nbx)));
-                    m1 = block_mask(sel1, min(8, g.fh - 8 * (i1 / g.nbx)), min(8, g.fw - 8 * (i1 % g.nbx)));
+                    m0 = sel0 ? blk_mask[L0 % g.nbf] : 0ull;
+                    m1 = sel1 ? blk_mask[L1 % g.nbf] : 0ull;
                 }
             };
             bool masked;
@@ -661,18 +671,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                 }
             }
             const float lse2 = (l > 0.f) ? m + fast_log2(l) : -CUDART_INF_F;
-            if (row_valid)
-                a.lse[(size_t)bh * a.q_frames * g.tf + qf * g.tf + qy * g.fw + qx] = lse2 * 0.6931471805599453f;
+            if (row_valid) a.lse[(size_t)bh * a.q_frames * g.tf + q_tok] = lse2 * 0.6931471805599453f;
             fence_proxy_async_smem();
             named_bar_sync(bar_id, 128);
             if (r == 0) {
                 for (int hb = 0; hb < 2; ++hb) {
                     const int qb = qblock(X, hb);
                     if (qb < 0) break;
-                    const int f = qb / g.nbf, i = qb % g.nbf;
+                    const BlockBox obb = block_box(g, qb % g.nbf);
+                    const int f0 = b * a.q_frames + (qb / g.nbf) * g.bt;
                     for (int hh = 0; hh < NH; ++hh)
-                        tma_store_5d(&a.tm_o, sO + hh * kHalf + hb * (kHalf / 2), hh * 64, h,
-                                     8 * (i % g.nbx), 8 * (i / g.nbx), b * a.q_frames + f);
+                        tma_store_5d(&a.tm_o, sO + hh * kHalf + hb * (kHalf / 2), hh * 64, h, obb.x0, obb.y0, f0);
                 }
                 tma_store_commit();
                 tma_store_wait_all();
@@ -700,9 +709,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                         if (a.mass_pers) atomicAdd(&a.mass_pers[(size_t)bh * S + seg_slot[sg]], v);
                     } else {
                         const int L = ublk[sg - n_occ];
-                        const int phys = (a.ring_head + L / g.nbf) % g.W;
+                        const int phys = (head_g + L / g.nbf) % g.Wg;
                         if (a.mass_local)
-                            atomicAdd(&a.mass_local[((size_t)bh * g.W + phys) * g.nbf + L % g.nbf], v);
+                            atomicAdd(&a.mass_local[((size_t)bh * g.Wg + phys) * g.nbf + L % g.nbf], v);
                     }
                 }
             }
@@ -734,14 +743,14 @@ cudaError_t launch_fwd_t(const FwdKernelArgs& ka, dim3 grid, size_t smem, cudaSt
 
 size_t attn_fwd_smem_bytes(const Geo& g, int ucap) {
     // at least 120 KB so that one CTA (holding all 512 TMEM columns) runs per SM
-    const size_t need = fwd_plan(g.D, g.S, ucap).total + 1024;
+    const size_t need = fwd_plan(g.D, g.S, ucap, g.nbf).total + 1024;
     return need < 120 * 1024 ? 120 * 1024 : need;
 }
 
 cudaError_t launch_attn_fwd(const FwdArgs& a, bool with_mass, cudaStream_t st) {
     FwdKernelArgs ka;
     ka.a = a;
-    ka.n_groups = (a.q_frames * a.g.nbf + 3) / 4;
+    ka.n_groups = (a.q_frames / a.g.bt * a.g.nbf + 3) / 4;
     const size_t smem = attn_fwd_smem_bytes(a.g, a.ucap);
     dim3 grid(ka.n_groups, a.g.H, a.g.B);
     if (a.g.D == 128)

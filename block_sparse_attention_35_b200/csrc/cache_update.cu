@@ -42,7 +42,8 @@ __global__ void __launch_bounds__(kMergeThreads) merge_rank_kernel(MergeParams p
     const Geo& g = p.g;
     const int S = g.S;
     const int h = blockIdx.x, b = blockIdx.y, bh = b * g.H + h;
-    const int n_ev = p.n_ev_frames * g.nbf;
+    const int n_ev = p.n_ev_frames / g.bt * g.nbf;
+    const int head_g = p.ring_head / g.bt;
     const int ncand_max = S + n_ev;
     float* sc = reinterpret_cast<float*>(smraw);            // [S + n_ev] candidate scores
     int* cid = reinterpret_cast<int*>(sc + ncand_max);      // [S + n_ev] slot or block id
@@ -83,8 +84,8 @@ __global__ void __launch_bounds__(kMergeThreads) merge_rank_kernel(MergeParams p
     const int n_occ = s_nocc;
     const int ncand = n_occ + n_ev;
     for (int j = threadIdx.x; j < n_ev; j += blockDim.x) {
-        const int phys = (p.ring_head + j / g.nbf) % g.W;
-        const size_t mi = ((size_t)bh * g.W + phys) * g.nbf + j % g.nbf;
+        const int phys = (head_g + j / g.nbf) % g.Wg;
+        const size_t mi = ((size_t)bh * g.Wg + phys) * g.nbf + j % g.nbf;
         cid[n_occ + j] = j;
         sc[n_occ + j] = p.mass_local[mi];
     }
@@ -124,10 +125,10 @@ __global__ void __launch_bounds__(kMergeThreads) merge_rank_kernel(MergeParams p
                 const int j = cid[c];
                 const int s = freel[k];
                 const int i = j % g.nbf;
-                const int hv = min(8, g.fh - 8 * (i / g.nbx)), wv = min(8, g.fw - 8 * (i % g.nbx));
-                p.pers_len[(size_t)bh * S + s] = hv * wv;
+                const BlockBox bb = block_box(g, i);
+                p.pers_len[(size_t)bh * S + s] = g.bt * bb.hv * bb.wv;
                 p.pers_score[(size_t)bh * S + s] = sc[c];
-                p.pers_src[(size_t)bh * S + s] = (p.first_frame_global + j / g.nbf) * g.nbf + i;
+                p.pers_src[(size_t)bh * S + s] = (p.first_frame_global / g.bt + j / g.nbf) * g.nbf + i;
                 p.upd[((size_t)bh * n_ev + k) * 2 + 0] = s;
                 p.upd[((size_t)bh * n_ev + k) * 2 + 1] = j;
             }
@@ -138,8 +139,8 @@ __global__ void __launch_bounds__(kMergeThreads) merge_rank_kernel(MergeParams p
     __syncthreads();
     // the evicted frames' slots of the ring start over for the next frames
     for (int j = threadIdx.x; j < n_ev; j += blockDim.x) {
-        const int phys = (p.ring_head + j / g.nbf) % g.W;
-        p.mass_local[((size_t)bh * g.W + phys) * g.nbf + j % g.nbf] = 0.f;
+        const int phys = (head_g + j / g.nbf) % g.Wg;
+        p.mass_local[((size_t)bh * g.Wg + phys) * g.nbf + j % g.nbf] = 0.f;
     }
 }
 
@@ -160,10 +161,11 @@ __global__ void __launch_bounds__(256) merge_copy_kernel(CopyParams p) {
     if (k >= p.n_upd[bh]) return;
     const int slot = p.upd[((size_t)bh * p.n_ev + k) * 2 + 0];
     const int j = p.upd[((size_t)bh * p.n_ev + k) * 2 + 1];
-    const int phys = (p.ring_head + j / g.nbf) % g.W;
-    const int i = j % g.nbf;
-    const int y0 = 8 * (i / g.nbx), x0 = 8 * (i % g.nbx);
-    const int hv = min(8, g.fh - y0), wv = min(8, g.fw - x0), c = hv * wv;
+    // first ring frame of the block's frame group (groups never wrap: W and ring_head are
+    // multiples of bt)
+    const int phys = (p.ring_head + (j / g.nbf) * g.bt) % g.W;
+    const BlockBox bb = block_box(g, j % g.nbf);
+    const int y0 = bb.y0, x0 = bb.x0, wv = bb.wv, plane = bb.hv * bb.wv, c = g.bt * plane;
     const int cpr = g.D / 8;  // 16-byte chunks per token row
     const size_t frame_base = ((size_t)b * g.W + phys) * g.tf;
     const size_t slot_base = ((size_t)bh * g.S + slot) * 64;
@@ -171,8 +173,8 @@ __global__ void __launch_bounds__(256) merge_copy_kernel(CopyParams p) {
         const int row = e / cpr, ch = e % cpr;
         uint4 kv = make_uint4(0, 0, 0, 0), vv = make_uint4(0, 0, 0, 0);
         if (row < c) {
-            const int y = y0 + row / wv, x = x0 + row % wv;
-            const size_t src = ((frame_base + (size_t)y * g.fw + x) * g.H + h) * g.D + ch * 8;
+            const int t = row / plane, y = y0 + (row % plane) / wv, x = x0 + row % wv;
+            const size_t src = ((frame_base + (size_t)t * g.tf + (size_t)y * g.fw + x) * g.H + h) * g.D + ch * 8;
             kv = __ldg(reinterpret_cast<const uint4*>(p.kl + src));
             vv = __ldg(reinterpret_cast<const uint4*>(p.vl + src));
         }
@@ -190,7 +192,7 @@ cudaError_t launch_cache_update(const Geo& g, const __nv_bfloat16* k_local,
                                 __nv_bfloat16* k_pers, __nv_bfloat16* v_pers, int32_t* pers_len,
                                 float* pers_score, int32_t* pers_src, int32_t* upd,
                                 int32_t* n_upd, cudaStream_t st) {
-    const int n_ev = n_evict_frames * g.nbf;
+    const int n_ev = n_evict_frames / g.bt * g.nbf;
     if (n_ev == 0) return cudaSuccess;
     MergeParams mp{g, local_frames, ring_head, n_evict_frames, first_frame_global,
                    mass_local, pers_len, pers_score, pers_src, upd, n_upd};

@@ -36,8 +36,9 @@ size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 int tokens_per_frame(const pbsa_config* c) { return c->frame_h * c->frame_w; }
 
+// blocks of one frame group (block_t frames)
 int blocks_per_frame(const pbsa_config* c) {
-    return ((c->frame_h + 7) / 8) * ((c->frame_w + 7) / 8);
+    return ((c->frame_h + c->block_h - 1) / c->block_h) * ((c->frame_w + c->block_w - 1) / c->block_w);
 }
 
 bool dense_mode(const pbsa_config* c) { return c->kv_cache_mode == PBSA_KV_CACHE_DENSE; }
@@ -47,13 +48,14 @@ int window_tokens(const pbsa_config* c) { return dense_mode(c) ? c->total_cache_
 
 int num_slots(const pbsa_config* c) {
     if (dense_mode(c)) return 0;
-    const int tf = tokens_per_frame(c);
-    if (c->persistent_cache_size % tf == 0) return c->persistent_cache_size / tf * blocks_per_frame(c);
-    return (c->persistent_cache_size + 63) / 64;
+    const int tg = tokens_per_frame(c) * c->block_t;
+    if (c->persistent_cache_size % tg == 0) return c->persistent_cache_size / tg * blocks_per_frame(c);
+    const int brows = c->block_t * c->block_h * c->block_w;
+    return (c->persistent_cache_size + brows - 1) / brows;
 }
 
 int topk_count(const pbsa_config* c, int local_frames) {
-    const int nl = local_frames * blocks_per_frame(c);
+    const int nl = local_frames / c->block_t * blocks_per_frame(c);
     if (nl <= 0) return 0;
     if (!c->use_local_block_sparse_attn || dense_mode(c)) return nl;
     const double k = std::ceil(static_cast<double>(c->local_block_sparse_topk_ratio) * nl);
@@ -70,28 +72,32 @@ int validate(const pbsa_config* c) {
     if (c->D != 64 && c->D != 128) return fail(PBSA_ERR_UNSUPPORTED, "head dim %d: only 64 and 128 are built", c->D);
     if (c->H * c->D > 8192) return fail(PBSA_ERR_UNSUPPORTED, "H*D = %d > 8192", c->H * c->D);
     if (c->frame_h < 1 || c->frame_w < 1) return fail(PBSA_ERR_ARG, "frame grid %dx%d", c->frame_h, c->frame_w);
-    if (c->block_t != 1 || c->block_h != 8 || c->block_w != 8)
-        return fail(PBSA_ERR_UNSUPPORTED, "sparse_kv_block_size [%d,%d,%d]: only [1,8,8] is built",
+    if (c->block_t < 1 || c->block_h < 1 || c->block_w < 1)
+        return fail(PBSA_ERR_ARG, "sparse_kv_block_size [%d,%d,%d]: sizes must be >= 1", c->block_t,
+                    c->block_h, c->block_w);
+    if (c->block_t * c->block_h * c->block_w > 64)
+        return fail(PBSA_ERR_UNSUPPORTED, "sparse_kv_block_size [%d,%d,%d]: blocks above 64 tokens are not built",
                     c->block_t, c->block_h, c->block_w);
     if (c->kv_cache_mode != PBSA_KV_CACHE_SPARSE_FORCING && c->kv_cache_mode != PBSA_KV_CACHE_DENSE)
         return fail(PBSA_ERR_UNSUPPORTED, "kv_cache_mode %d: only sparse_forcing and dense are built",
                     c->kv_cache_mode);
     const int tf = tokens_per_frame(c);
-    if (c->local_cache_size < tf || c->local_cache_size % tf)
-        return fail(PBSA_ERR_ARG, "local_cache_size %d is not a positive multiple of %d tokens/frame",
-                    c->local_cache_size, tf);
-    if (dense_mode(c) && c->total_cache_size % tf)
-        return fail(PBSA_ERR_ARG, "dense mode: total_cache_size %d is not a multiple of %d tokens/frame",
-                    c->total_cache_size, tf);
+    const int tg = tf * c->block_t;   // a frame group: the frames one block spans
+    if (c->local_cache_size < tg || c->local_cache_size % tg)
+        return fail(PBSA_ERR_ARG, "local_cache_size %d is not a positive multiple of %d tokens (%d frame(s))",
+                    c->local_cache_size, tg, c->block_t);
+    if (dense_mode(c) && c->total_cache_size % tg)
+        return fail(PBSA_ERR_ARG, "dense mode: total_cache_size %d is not a multiple of %d tokens",
+                    c->total_cache_size, tg);
     if (c->persistent_cache_size < 0) return fail(PBSA_ERR_ARG, "persistent_cache_size < 0");
     if (c->total_cache_size != c->local_cache_size + c->persistent_cache_size)
         return fail(PBSA_ERR_ARG, "total_cache_size %d != local %d + persistent %d",
                     c->total_cache_size, c->local_cache_size, c->persistent_cache_size);
-    if (c->max_seq_len < tf) return fail(PBSA_ERR_ARG, "max_seq_len %d < one frame (%d)", c->max_seq_len, tf);
+    if (c->max_seq_len < tg) return fail(PBSA_ERR_ARG, "max_seq_len %d < one frame group (%d)", c->max_seq_len, tg);
     const float r = c->local_block_sparse_topk_ratio;
     if (!(r > 0.f && r <= 1.f)) return fail(PBSA_ERR_ARG, "local_block_sparse_topk_ratio %g not in (0, 1]", r);
     const int W = window_tokens(c) / tf;
-    const int nlmax = W * blocks_per_frame(c);
+    const int nlmax = W / c->block_t * blocks_per_frame(c);
     if (nlmax > 512) return fail(PBSA_ERR_UNSUPPORTED, "%d local blocks > 512", nlmax);
     if (num_slots(c) > 1024) return fail(PBSA_ERR_UNSUPPORTED, "%d persistent slots > 1024", num_slots(c));
     return PBSA_OK;
@@ -105,10 +111,15 @@ pbsa::Geo make_geo(const pbsa_config* c) {
     g.fh = c->frame_h;
     g.fw = c->frame_w;
     g.tf = c->frame_h * c->frame_w;
-    g.nby = (c->frame_h + 7) / 8;
-    g.nbx = (c->frame_w + 7) / 8;
+    g.bt = c->block_t;
+    g.bh = c->block_h;
+    g.bw = c->block_w;
+    g.brows = g.bt * g.bh * g.bw;
+    g.nby = (c->frame_h + g.bh - 1) / g.bh;
+    g.nbx = (c->frame_w + g.bw - 1) / g.bw;
     g.nbf = g.nby * g.nbx;
     g.W = window_tokens(c) / g.tf;
+    g.Wg = g.W / g.bt;
     g.S = num_slots(c);
     return g;
 }
@@ -120,6 +131,9 @@ int check_window(const pbsa_config* c, const pbsa::Geo& g, int q_frames, int loc
     if (local_frames < 1 || local_frames > g.W)
         return fail(PBSA_ERR_ARG, "local_frames %d not in [1, %d]", local_frames, g.W);
     if (ring_head < 0 || ring_head >= g.W) return fail(PBSA_ERR_ARG, "ring_head %d not in [0, %d)", ring_head, g.W);
+    if (q_frames % g.bt || local_frames % g.bt || ring_head % g.bt)
+        return fail(PBSA_ERR_ARG, "q_frames %d, local_frames %d and ring_head %d must be multiples of block_t %d",
+                    q_frames, local_frames, ring_head, g.bt);
     return PBSA_OK;
 }
 
@@ -154,7 +168,8 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-// [frames, frame_h, frame_w, H, D] bf16 tensor, box [1, 8, 8, 1, 64], 128-byte swizzle.
+// [frames, frame_h, frame_w, H, D] bf16 tensor, box [bt, bh, bw, 1, 64] (one block, its rows
+// in frame / row / column order), 128-byte swizzle.
 int map_tokens(CUtensorMap* m, const void* ptr, const pbsa::Geo& g, long long frames) {
     auto enc = encode_fn();
     if (!enc) return fail(PBSA_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
@@ -162,7 +177,7 @@ int map_tokens(CUtensorMap* m, const void* ptr, const pbsa::Geo& g, long long fr
                           (cuuint64_t)frames};
     cuuint64_t strides[4] = {(cuuint64_t)g.D * 2, (cuuint64_t)g.H * g.D * 2,
                              (cuuint64_t)g.fw * g.H * g.D * 2, (cuuint64_t)g.fh * g.fw * g.H * g.D * 2};
-    cuuint32_t box[5] = {64, 1, 8, 8, 1};
+    cuuint32_t box[5] = {64, 1, (cuuint32_t)g.bw, (cuuint32_t)g.bh, (cuuint32_t)g.bt};
     cuuint32_t es[5] = {1, 1, 1, 1, 1};
     CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(ptr), dims, strides, box, es,
                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -201,8 +216,8 @@ int map_slots(CUtensorMap* m8, CUtensorMap* m64, const void* pers, const void* w
 }
 
 size_t select_ws(const pbsa::Geo& g, int q_frames) {
-    return align256(sizeof(float) * (size_t)g.B * g.H * q_frames * g.nbf * g.D) +
-           align256(sizeof(float) * (size_t)g.B * g.H * g.W * g.nbf * g.D);
+    return align256(sizeof(float) * (size_t)g.B * g.H * (q_frames / g.bt) * g.nbf * g.D) +
+           align256(sizeof(float) * (size_t)g.B * g.H * g.Wg * g.nbf * g.D);
 }
 
 int fwd_ucap(const pbsa_config* c, const pbsa::Geo& g, int idx_stride) {
@@ -212,7 +227,7 @@ int fwd_ucap(const pbsa_config* c, const pbsa::Geo& g, int idx_stride) {
 
 size_t fwd_ws(const pbsa_config* c, const pbsa::Geo& g, int q_frames) {
     // per CTA of four query blocks, two 128-row sides
-    const size_t ctas = (size_t)g.B * g.H * 2 * ((q_frames * g.nbf + 3) / 4);
+    const size_t ctas = (size_t)g.B * g.H * 2 * ((q_frames / g.bt * g.nbf + 3) / 4);
     const size_t nseg = (size_t)g.S + 2 * topk_count(c, g.W);
     return align256(sizeof(float) * ctas * nseg * 128);
 }
@@ -268,38 +283,28 @@ size_t pbsa_workspace_size(const pbsa_config* cfg, int op, int q_frames) {
 int pbsa_select_blocks(const pbsa_config* cfg, const void* q, int q_frames, const void* k_local,
                        int local_frames, int ring_head, int32_t* idx, int idx_stride, int32_t* cnt,
                        float* scores, void* workspace, size_t workspace_bytes, void* stream) {
-    int rc = validate(cfg);
+    pbsa::Geo g;
+    int k = 0;
+    size_t need = 0, key_off = 0;
+    int rc = pbsa::api_prepare_select(cfg, q, q_frames, k_local, local_frames, ring_head, idx, idx_stride,
+                                      cnt, scores, &g, &k, &need, &key_off);
     if (rc != PBSA_OK) return rc;
-    const pbsa::Geo g = make_geo(cfg);
-    if ((rc = check_window(cfg, g, q_frames, local_frames, ring_head)) != PBSA_OK) return rc;
-    REQUIRE_PTR(q);
-    REQUIRE_PTR(k_local);
-    REQUIRE_PTR(idx);
-    REQUIRE_PTR(cnt);
-    OPTIONAL_PTR(scores);
-    REQUIRE_PTR(workspace);
-    const int k = topk_count(cfg, local_frames);
-    if (idx_stride < k) return fail(PBSA_ERR_ARG, "idx_stride %d < k %d", idx_stride, k);
-    const size_t need = select_ws(g, q_frames);
-    if (workspace_bytes < need)
-        return fail(PBSA_ERR_WORKSPACE, "workspace %zu < %zu bytes", workspace_bytes, need);
-    const int nl = local_frames * g.nbf;
-    if (pbsa::score_topk_smem_bytes(g, nl) > 227 * 1024)
-        return fail(PBSA_ERR_UNSUPPORTED, "%d local blocks do not fit the scoring kernel", nl);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (k == nl && !scores) {
-        cudaError_t e = pbsa::launch_select_all(g, q_frames * g.nbf, nl, idx, idx_stride, cnt, st);
+    const int qb = q_frames / g.bt * g.nbf, nl = local_frames / g.bt * g.nbf;
+    if (k == nl && !scores) {   // every window block, no scores: no pooling, no workspace
+        cudaError_t e = pbsa::launch_select_all(g, qb, nl, idx, idx_stride, cnt, st);
         if (e != cudaSuccess) return cuda_fail(e, "select-all kernel launch");
         return PBSA_OK;
     }
+    REQUIRE_PTR(workspace);
+    if (workspace_bytes < need) return fail(PBSA_ERR_WORKSPACE, "workspace %zu < %zu bytes", workspace_bytes, need);
     float* qbar = static_cast<float*>(workspace);
-    float* kbar = reinterpret_cast<float*>(static_cast<char*>(workspace) +
-                                           align256(sizeof(float) * (size_t)g.B * g.H * q_frames * g.nbf * g.D));
+    float* kbar = reinterpret_cast<float*>(static_cast<char*>(workspace) + key_off);
     cudaError_t e = pbsa::launch_pool(g, static_cast<const __nv_bfloat16*>(q), q_frames,
                                       static_cast<const __nv_bfloat16*>(k_local), ring_head, local_frames,
                                       qbar, kbar, st);
     if (e != cudaSuccess) return cuda_fail(e, "pool kernel launch");
-    e = pbsa::launch_score_topk(g, qbar, kbar, ring_head, q_frames * g.nbf, nl, k, idx, idx_stride, cnt, scores, st);
+    e = pbsa::launch_score_topk(g, qbar, kbar, ring_head, qb, nl, k, idx, idx_stride, cnt, scores, st);
     if (e != cudaSuccess) return cuda_fail(e, "score/top-k kernel launch");
     return PBSA_OK;
 }
@@ -311,6 +316,9 @@ int pbsa_pool_keys(const pbsa_config* cfg, const void* k_local, int first_slot, 
     const pbsa::Geo g = make_geo(cfg);
     if (first_slot < 0 || first_slot >= g.W) return fail(PBSA_ERR_ARG, "first_slot %d not in [0, %d)", first_slot, g.W);
     if (n_frames < 0 || n_frames > g.W) return fail(PBSA_ERR_ARG, "n_frames %d not in [0, %d]", n_frames, g.W);
+    if (first_slot % g.bt || n_frames % g.bt)
+        return fail(PBSA_ERR_ARG, "first_slot %d and n_frames %d must be multiples of block_t %d", first_slot,
+                    n_frames, g.bt);
     REQUIRE_PTR(k_local);
     REQUIRE_PTR(kbar);
     cudaError_t e = pbsa::launch_pool(g, nullptr, 0, static_cast<const __nv_bfloat16*>(k_local), first_slot,
@@ -333,15 +341,15 @@ int pbsa_select_blocks_pooled(const pbsa_config* cfg, const void* q, int q_frame
     OPTIONAL_PTR(scores);
     const int k = topk_count(cfg, local_frames);
     if (idx_stride < k) return fail(PBSA_ERR_ARG, "idx_stride %d < k %d", idx_stride, k);
-    const int nl = local_frames * g.nbf;
+    const int nl = local_frames / g.bt * g.nbf;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (k == nl && !scores) {
-        cudaError_t e = pbsa::launch_select_all(g, q_frames * g.nbf, nl, idx, idx_stride, cnt, st);
+        cudaError_t e = pbsa::launch_select_all(g, q_frames / g.bt * g.nbf, nl, idx, idx_stride, cnt, st);
         if (e != cudaSuccess) return cuda_fail(e, "select-all kernel launch");
         return PBSA_OK;
     }
     REQUIRE_PTR(workspace);
-    const size_t need = align256(sizeof(float) * (size_t)g.B * g.H * q_frames * g.nbf * g.D);
+    const size_t need = align256(sizeof(float) * (size_t)g.B * g.H * (q_frames / g.bt) * g.nbf * g.D);
     if (workspace_bytes < need) return fail(PBSA_ERR_WORKSPACE, "workspace %zu < %zu bytes", workspace_bytes, need);
     if (pbsa::score_topk_smem_bytes(g, nl) > 227 * 1024)
         return fail(PBSA_ERR_UNSUPPORTED, "%d local blocks do not fit the scoring kernel", nl);
@@ -349,7 +357,7 @@ int pbsa_select_blocks_pooled(const pbsa_config* cfg, const void* q, int q_frame
     cudaError_t e = pbsa::launch_pool(g, static_cast<const __nv_bfloat16*>(q), q_frames, nullptr, 0, 0, qbar,
                                       nullptr, st);
     if (e != cudaSuccess) return cuda_fail(e, "pool kernel launch");
-    e = pbsa::launch_score_topk(g, qbar, kbar, ring_head, q_frames * g.nbf, nl, k, idx, idx_stride, cnt, scores, st);
+    e = pbsa::launch_score_topk(g, qbar, kbar, ring_head, q_frames / g.bt * g.nbf, nl, k, idx, idx_stride, cnt, scores, st);
     if (e != cudaSuccess) return cuda_fail(e, "score/top-k kernel launch");
     return PBSA_OK;
 }
@@ -487,10 +495,13 @@ int pbsa_cache_update(const pbsa_config* cfg, const void* k_local, const void* v
     int rc = validate(cfg);
     if (rc != PBSA_OK) return rc;
     const pbsa::Geo g = make_geo(cfg);
-    if ((rc = check_window(cfg, g, 1, local_frames, ring_head)) != PBSA_OK) return rc;
+    if ((rc = check_window(cfg, g, g.bt, local_frames, ring_head)) != PBSA_OK) return rc;
     if (n_evict_frames < 0 || n_evict_frames > local_frames)
         return fail(PBSA_ERR_ARG, "n_evict_frames %d not in [0, local_frames=%d]", n_evict_frames, local_frames);
     if (first_frame_global < 0) return fail(PBSA_ERR_ARG, "first_frame_global < 0");
+    if (n_evict_frames % g.bt || first_frame_global % g.bt)
+        return fail(PBSA_ERR_ARG, "n_evict_frames %d and first_frame_global %d must be multiples of block_t %d",
+                    n_evict_frames, first_frame_global, g.bt);
     REQUIRE_PTR(k_local);
     REQUIRE_PTR(v_local);
     REQUIRE_PTR(mass_local);
@@ -546,13 +557,13 @@ int api_prepare_select(const pbsa_config* cfg, const void* q, int q_frames, cons
     OPTIONAL_PTR(scores);
     const int kk = topk_count(cfg, local_frames);
     if (idx_stride < kk) return fail(PBSA_ERR_ARG, "idx_stride %d < k %d", idx_stride, kk);
-    const int nl = local_frames * g.nbf;
+    const int nl = local_frames / g.bt * g.nbf;
     if (score_topk_smem_bytes(g, nl) > 227 * 1024)
         return fail(PBSA_ERR_UNSUPPORTED, "%d local blocks do not fit the scoring kernel", nl);
     *geo = g;
     *k = kk;
     *scratch_bytes = select_ws(g, q_frames);
-    *key_offset = align256(sizeof(float) * (size_t)g.B * g.H * q_frames * g.nbf * g.D);
+    *key_offset = align256(sizeof(float) * (size_t)g.B * g.H * (q_frames / g.bt) * g.nbf * g.D);
     return PBSA_OK;
 }
 

@@ -12,13 +12,55 @@
 namespace pbsa {
 
 // Geometry derived from a pbsa_config (all counts in tokens, blocks or frames).
+// A block is bt x bh x bw tokens (sparse_kv_block_size): bt consecutive frames ("a frame
+// group") x bh rows x bw columns; edge blocks are clipped to the frame.  Block ids count
+// frame groups: id = group * nbf + block in group.  Every frame count the ABI takes is a
+// multiple of bt.
 struct Geo {
     int B, H, D;
     int fh, fw, tf;     // frame grid and tokens per frame
-    int nby, nbx, nbf;  // block rows, block columns, blocks per frame
+    int bt, bh, bw;     // block shape (frames, rows, columns)
+    int brows;          // bt * bh * bw: rows of a full block (<= 64)
+    int nby, nbx, nbf;  // block rows, block columns, blocks per frame group
     int W;              // frame slots of the local ring
+    int Wg;             // frame groups of the ring (W / bt)
     int S;              // persistent slots
 };
+
+// Block i of a frame group: first row and column in the frame and its valid extent.
+struct BlockBox {
+    int y0, x0, hv, wv;
+};
+
+__host__ __device__ inline BlockBox block_box(const Geo& g, int i) {
+    BlockBox b;
+    b.y0 = g.bh * (i / g.nbx);
+    b.x0 = g.bw * (i % g.nbx);
+    b.hv = min(g.bh, g.fh - b.y0);
+    b.wv = min(g.bw, g.fw - b.x0);
+    return b;
+}
+
+// Row r (0..63) of a block as a TMA box lays it out (column fastest, then row, then frame):
+// frame t, row y, column x inside the block; true when the token exists (r < brows and
+// inside the frame).
+__host__ __device__ inline bool block_row(const Geo& g, const BlockBox& bb, int r, int* t, int* y, int* x) {
+    *x = r % g.bw;
+    *y = (r / g.bw) % g.bh;
+    *t = r / (g.bw * g.bh);
+    return r < g.brows && *y < bb.hv && *x < bb.wv;
+}
+
+// Valid rows of block i as a 64-bit mask over its box rows.
+__host__ __device__ inline uint64_t block_rows_mask(const Geo& g, int i) {
+    const BlockBox bb = block_box(g, i);
+    uint64_t m = 0;
+    for (int r = 0; r < g.brows; ++r) {
+        int t, y, x;
+        if (block_row(g, bb, r, &t, &y, &x)) m |= 1ull << r;
+    }
+    return m;
+}
 
 // Forward-pass launch arguments.
 struct FwdArgs {

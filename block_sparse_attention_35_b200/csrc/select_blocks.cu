@@ -8,11 +8,12 @@
 //
 // Two kernels:
 //  1. pool_kernel: one CTA per (block, batch); each thread owns 8 consecutive channels of
-//     the token's [H, D] row and streams the block's valid tokens with 16-byte loads, so a
-//     CTA reads whole 3 KB token rows (all heads) - fully coalesced, one HBM pass over Q
-//     and the window's K.  Means go to fp32 workspace; key means are stored by physical
-//     ring slot, so a caller can keep them across chunks and pool only the frames it
-//     appends (pbsa_pool_keys + pbsa_select_blocks_pooled).
+//     the token's [H, D] row and streams the block's valid tokens (all bt frames of its
+//     frame group) with 16-byte loads, so a CTA reads whole 3 KB token rows (all heads) -
+//     fully coalesced, one HBM pass over Q and the window's K.  Means go to fp32
+//     workspace; key means are stored by physical ring frame group, so a caller can keep
+//     them across chunks and pool only the frames it appends (pbsa_pool_keys +
+//     pbsa_select_blocks_pooled).
 //  2. score_topk_kernel: one CTA per (8 query blocks, head, batch); the head's pooled keys
 //     sit in shared memory (rows padded to D+1 floats: conflict-free), one warp per query
 //     block computes its N_L scores, ranks every candidate by counting the candidates that
@@ -32,14 +33,14 @@ struct PoolParams {
     const __nv_bfloat16* q;
     const __nv_bfloat16* kl;
     int q_frames;           // query frames to pool (0: none)
-    int k_first, k_frames;  // ring slots k_first, k_first+1, ... (mod W) of K to pool
+    int k_first, k_frames;  // ring frames k_first, k_first+1, ... (mod W) of K to pool
     float* qbar;  // [B, H, QB, D]
-    float* kbar;  // [B, H, W*NB_f, D], by physical ring slot
+    float* kbar;  // [B, H, Wg*NB, D], by physical ring frame group
 };
 
 __global__ void __launch_bounds__(1024) pool_kernel(PoolParams p) {
     const Geo& g = p.g;
-    const int qb_total = p.q_frames * g.nbf;
+    const int qb_total = p.q_frames / g.bt * g.nbf;
     const int blk = blockIdx.x;
     const int b = blockIdx.y;
     const int hd = g.H * g.D;
@@ -47,31 +48,31 @@ __global__ void __launch_bounds__(1024) pool_kernel(PoolParams p) {
     if (t * 8 >= hd) return;
 
     const __nv_bfloat16* src;
-    long long frame;  // frame index inside the source tensor
+    long long frame;  // first frame of the block's group inside the source tensor
     int i_in_frame;
     float* dst;
     int local_id, n_of_kind;
     if (blk < qb_total) {
-        frame = (long long)b * p.q_frames + blk / g.nbf;
+        frame = (long long)b * p.q_frames + (long long)(blk / g.nbf) * g.bt;
         i_in_frame = blk % g.nbf;
         src = p.q;
         dst = p.qbar;
         local_id = blk;
         n_of_kind = qb_total;
     } else {
-        const int j = blk - qb_total;  // j-th block of the K frames being pooled
-        const int phys = (p.k_first + j / g.nbf) % g.W;
-        frame = (long long)b * g.W + phys;
+        const int j = blk - qb_total;  // j-th block of the K frame groups being pooled
+        const int phys = (p.k_first / g.bt + j / g.nbf) % g.Wg;
+        frame = (long long)b * g.W + (long long)phys * g.bt;
         i_in_frame = j % g.nbf;
         src = p.kl;
         dst = p.kbar;
         local_id = phys * g.nbf + i_in_frame;
-        n_of_kind = g.W * g.nbf;
+        n_of_kind = g.Wg * g.nbf;
     }
-    const int by = i_in_frame / g.nbx, bx = i_in_frame % g.nbx;
-    const int y0 = by * 8, x0 = bx * 8;
-    const int hv = min(8, g.fh - y0), wv = min(8, g.fw - x0);
-    const int n = hv * wv;
+    const BlockBox bb = block_box(g, i_in_frame);
+    const int y0 = bb.y0, x0 = bb.x0, hv = bb.hv, wv = bb.wv;
+    const int plane = hv * wv;
+    const int n = g.bt * plane;
 
     float acc[8];
 #pragma unroll
@@ -84,8 +85,8 @@ __global__ void __launch_bounds__(1024) pool_kernel(PoolParams p) {
         for (int u = 0; u < 8; ++u) {
             const int r = r0 + u;
             if (r < n) {
-                const int y = y0 + r / wv, x = x0 + r % wv;
-                v[u] = __ldg(reinterpret_cast<const uint4*>(base + (long long)(y * g.fw + x) * hd));
+                const int t = r / plane, y = y0 + (r % plane) / wv, x = x0 + r % wv;
+                v[u] = __ldg(reinterpret_cast<const uint4*>(base + ((long long)t * g.tf + y * g.fw + x) * hd));
             }
         }
 #pragma unroll
@@ -116,7 +117,7 @@ constexpr int kMaxChunks = 16; // candidates per warp lane: N_L <= 512
 struct ScoreParams {
     Geo g;
     const float* qbar;
-    const float* kbar;  // [B, H, W*NB_f, D] by physical ring slot
+    const float* kbar;  // [B, H, Wg*NB, D] by physical ring frame group
     int ring_head;
     int qb_total, nl, k;
     int32_t* idx;
@@ -138,13 +139,15 @@ __global__ void __launch_bounds__(256) score_topk_kernel(ScoreParams p) {
 
     // 16-byte loads, several in flight per thread (the copy is latency-bound otherwise);
     // rows are stored padded to D + 1 floats so that the dot products below are conflict-free
-    // logical window block j (oldest frame first) is ring row ((ring_head + j / NB_f) % W, j % NB_f)
-    const float* kbh = p.kbar + (size_t)bh * g.W * g.nbf * D;
+    // logical window block j (oldest frame group first) is ring row
+    // ((ring_head / bt + j / NB) % Wg, j % NB)
+    const float* kbh = p.kbar + (size_t)bh * g.Wg * g.nbf * D;
     const int n4 = nl * D / 4;
+    const int head_g = p.ring_head / g.bt;
 #pragma unroll 4
     for (int e = threadIdx.x; e < n4; e += blockDim.x) {
         const int j = (4 * e) / D, d = (4 * e) % D;
-        const int row = ((p.ring_head + j / g.nbf) % g.W) * g.nbf + j % g.nbf;
+        const int row = ((head_g + j / g.nbf) % g.Wg) * g.nbf + j % g.nbf;
         const float4 v = __ldg(reinterpret_cast<const float4*>(kbh + (size_t)row * D + d));
         float* dst = kb + j * (D + 1) + d;
         dst[0] = v.x;
@@ -235,7 +238,7 @@ cudaError_t launch_pool(const Geo& g, const __nv_bfloat16* q, int q_frames,
                         const __nv_bfloat16* k_local, int k_first, int k_frames,
                         float* qbar, float* kbar, cudaStream_t st) {
     PoolParams p{g, q, k_local, q_frames, k_first, k_frames, qbar, kbar};
-    const int nblk = (q_frames + k_frames) * g.nbf;
+    const int nblk = (q_frames + k_frames) / g.bt * g.nbf;
     if (nblk == 0) return cudaSuccess;
     const int threads = (g.H * g.D / 8 + 31) / 32 * 32;
     pool_kernel<<<dim3(nblk, g.B), threads, 0, st>>>(p);

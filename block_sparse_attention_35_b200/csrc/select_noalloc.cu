@@ -57,8 +57,8 @@ extern "C" PBSA_API int pbsa_select_blocks_noalloc(const pbsa_config* cfg, const
                                       cnt, scores, &g, &k, &need, &key_off);
     if (rc != PBSA_OK) return rc;
     // every window block selected and no scores asked for: no scratch needed
-    if (k == local_frames * g.nbf && !scores) {
-        cudaError_t e = pbsa::launch_select_all(g, q_frames * g.nbf, k, idx, idx_stride, cnt,
+    if (k == local_frames / g.bt * g.nbf && !scores) {
+        cudaError_t e = pbsa::launch_select_all(g, q_frames / g.bt * g.nbf, k, idx, idx_stride, cnt,
                                                 static_cast<cudaStream_t>(stream));
         if (e != cudaSuccess) return pbsa::api_cuda_fail(e, "select-all kernel launch");
         return PBSA_OK;
@@ -78,7 +78,7 @@ extern "C" PBSA_API int pbsa_select_blocks_noalloc(const pbsa_config* cfg, const
                                       static_cast<const __nv_bfloat16*>(k_local), ring_head, local_frames,
                                       qbar, kbar, st);
     if (e != cudaSuccess) return pbsa::api_cuda_fail(e, "pool kernel launch");
-    e = pbsa::launch_score_topk(g, qbar, kbar, ring_head, q_frames * g.nbf, local_frames * g.nbf, k, idx, idx_stride,
+    e = pbsa::launch_score_topk(g, qbar, kbar, ring_head, q_frames / g.bt * g.nbf, local_frames / g.bt * g.nbf, k, idx, idx_stride,
                                 cnt, scores, st);
     if (e != cudaSuccess) return pbsa::api_cuda_fail(e, "score/top-k kernel launch");
     return PBSA_OK;

@@ -71,6 +71,12 @@ WORKLOADS = {
                        local_cache_size=9360, persistent_cache_size=9360,
                        total_cache_size=18720, max_seq_len=32760, q_frames=3,
                        topk_ratio=0.125, bias_fraction=0.05, seed=1),
+    # The page-sized decode step with the project page's [3,4,4] blocks (3 frames x 4 x 4
+    # tokens): 104 blocks per 3-frame group, 208 slots, 208 window blocks, k = 26.
+    "decode344": Workload("decode344", B=1, H=12, D=128, frame_h=30, frame_w=52,
+                          local_cache_size=9360, persistent_cache_size=9360,
+                          total_cache_size=18720, max_seq_len=32760, q_frames=3,
+                          topk_ratio=0.125, block=(3, 4, 4), bias_fraction=0.05, seed=4),
     # Rollout: decode shapes, 20 chunks, empty persistent cache at the start.
     "rollout": Workload("rollout", B=1, H=12, D=128, frame_h=30, frame_w=52,
                         local_cache_size=9360, persistent_cache_size=9360,
@@ -88,7 +94,8 @@ def block_extents(frame_h: int, frame_w: int, bh: int = 8, bw: int = 8):
     """(rows, cols) of every block of one frame, in block order (row of blocks, then column).
 
     Edge blocks are clipped to the frame, so a 30x52 frame has 8x8, 8x4, 6x8 and 6x4
-    blocks.  Used only to lay out the synthetic persistent store.
+    blocks.  A block of bt frames has bt * rows * cols tokens.  Used only to lay out the
+    synthetic persistent store and the biased blocks.
     """
     out = []
     for y0 in range(0, frame_h, bh):
@@ -99,11 +106,12 @@ def block_extents(frame_h: int, frame_w: int, bh: int = 8, bw: int = 8):
 
 def slot_count(wl: Workload) -> int:
     """Number of 64-row persistent slots for the workload's persistent_cache_size."""
-    tf = wl.tokens_per_frame
+    bt = wl.block[0]
+    tg = wl.tokens_per_frame * bt
     nbf = len(block_extents(wl.frame_h, wl.frame_w, wl.block[1], wl.block[2]))
-    if wl.persistent_cache_size % tf == 0:
-        return wl.persistent_cache_size // tf * nbf
-    cap = wl.block[1] * wl.block[2]
+    if wl.persistent_cache_size % tg == 0:
+        return wl.persistent_cache_size // tg * nbf
+    cap = bt * wl.block[1] * wl.block[2]
     return -(-wl.persistent_cache_size // cap)
 
 
@@ -124,10 +132,10 @@ def _bias_local(gen, x, wl, frames):
     """
     if wl.bias_fraction <= 0:
         return
-    bh, bw = wl.block[1], wl.block[2]
+    bt, bh, bw = wl.block
     ext = block_extents(wl.frame_h, wl.frame_w, bh, bw)
     nbx = -(-wl.frame_w // bw)
-    nblk = frames * len(ext)
+    nblk = frames // bt * len(ext)
     nb = int(round(wl.bias_fraction * nblk))
     xv = x.view(wl.B, frames, wl.frame_h, wl.frame_w, wl.H, wl.D)
     for b in range(wl.B):
@@ -137,20 +145,19 @@ def _bias_local(gen, x, wl, frames):
             for j in pick:
                 f, i = divmod(j, len(ext))
                 by, bx = divmod(i, nbx)
-                xv[b, f, by * bh:by * bh + bh, bx * bw:bx * bw + bw, h, :] += u
+                xv[b, f * bt:f * bt + bt, by * bh:by * bh + bh, bx * bw:bx * bw + bw, h, :] += u
 
 
 def _persistent(gen, wl, n_slots, filled_slots):
     """Persistent store [B,H,S,64,D] whose first filled_slots slots hold blocks with the
     frame's block-size pattern; rows past each slot's length are zero."""
     ext = block_extents(wl.frame_h, wl.frame_w, wl.block[1], wl.block[2])
-    cap = wl.block[1] * wl.block[2]
-    k = torch.zeros(wl.B, wl.H, n_slots, cap, wl.D)
-    v = torch.zeros(wl.B, wl.H, n_slots, cap, wl.D)
+    k = torch.zeros(wl.B, wl.H, n_slots, 64, wl.D)
+    v = torch.zeros(wl.B, wl.H, n_slots, 64, wl.D)
     length = torch.zeros(wl.B, wl.H, n_slots, dtype=torch.int32)
     for s in range(filled_slots):
         r, c = ext[s % len(ext)]
-        length[:, :, s] = r * c
+        length[:, :, s] = wl.block[0] * r * c
     for b in range(wl.B):
         for h in range(wl.H):
             for s in range(filled_slots):

@@ -5,7 +5,7 @@
  * PBSA is the attention of "Sparse Forcing: Native Trainable Sparse Attention for
  * Real-time Autoregressive Diffusion Video Generation" (pith.science, abstract): a chunk of
  * video query tokens attends to every block of a persistent cache and to a top-k
- * selection of the 1x8x8 token blocks of a sliding local window; when the window slides,
+ * selection of the token blocks (1x8x8 or 3x4x4) of a sliding local window; when the window slides,
  * the evicted blocks are merged into the persistent cache.  The argument names follow the
  * project page's usage snippet of SparseForcingAttention (boxunxu.top/SparseForcing):
  * total_cache_size, local_cache_size, persistent_cache_size, kv_cache_mode,
@@ -41,12 +41,19 @@
  *                            zero): the kernels stream slots in 8-row groups and multiply
  *                            the masked rows by an exact zero.
  *      pers_len [B, H, S] int32 (0 = empty slot, else the block's token count, 1..64:
- *                            64 for an interior 8x8 block, hv * wv for a block cut by
- *                            the frame edge, e.g. 6 x 2 = 12 on a 30 x 50 grid).
- *  - Blocks: 1 x 8 x 8 tokens; a frame has NB_f = ceil(frame_h/8) * ceil(frame_w/8)
- *    blocks numbered by * ceil(frame_w/8) + bx; edge blocks are clipped to the frame.
- *    Local block ids are LOGICAL: window frame p, block i -> p * NB_f + i.  Query block
- *    ids: chunk frame f, block i -> f * NB_f + i.
+ *                            block_t * block_h * block_w for an interior block,
+ *                            block_t * hv * wv for a block cut by the frame edge, e.g.
+ *                            6 x 2 = 12 for [1,8,8] on a 30 x 50 grid).
+ *  - Blocks (sparse_kv_block_size = [block_t, block_h, block_w], e.g. [1, 8, 8] or the
+ *    project page's [3, 4, 4]): block_t consecutive frames (a "frame group") x block_h
+ *    rows x block_w columns.  A frame group has NB = ceil(frame_h / block_h) *
+ *    ceil(frame_w / block_w) blocks numbered by * ceil(frame_w / block_w) + bx; edge
+ *    blocks are clipped to the frame.  Inside a block (and in a persistent slot) tokens
+ *    are listed frame by frame, each frame in raster order.  Local block ids are LOGICAL:
+ *    window frame group p, block i -> p * NB + i.  Query block ids: chunk frame group f,
+ *    block i -> f * NB + i.  Every frame count and frame position the calls take
+ *    (q_frames, local_frames, ring_head, n_evict_frames, first_frame_global, ...) must be
+ *    a multiple of block_t, and so must the window (local_cache_size / T_f).
  */
 #ifndef PBSA_H
 #define PBSA_H
@@ -93,7 +100,7 @@ extern "C" {
 typedef struct pbsa_config {
     int B, H, D;                 /* batch, heads, head dim (64 or 128) */
     int frame_h, frame_w;        /* token grid of one frame, e.g. 30 x 52 */
-    int block_t, block_h, block_w; /* sparse_kv_block_size; only {1, 8, 8} is built */
+    int block_t, block_h, block_w; /* sparse_kv_block_size; block_t*block_h*block_w <= 64 */
     int total_cache_size;        /* tokens; must equal local + persistent */
     int local_cache_size;        /* tokens; a whole number of frames */
     int persistent_cache_size;   /* tokens */
@@ -107,16 +114,16 @@ typedef struct pbsa_config {
 
 /* Checks a configuration; PBSA_OK or an error code (message in pbsa_last_error()). */
 PBSA_API int pbsa_validate_config(const pbsa_config* cfg);
-/* NB_f, blocks per frame. */
+/* NB, blocks per frame group (per frame when block_t = 1). */
 PBSA_API int pbsa_blocks_per_frame(const pbsa_config* cfg);
 /* W, frame slots of the local ring (local_cache_size / T_f; total_cache_size / T_f in
  * dense mode). */
 PBSA_API int pbsa_window_frames(const pbsa_config* cfg);
-/* S, persistent slots: persistent_cache_size / T_f * NB_f when that divides, else
- * ceil(persistent_cache_size / 64); 0 in dense mode. */
+/* S, persistent slots: persistent_cache_size / (block_t * T_f) * NB when that divides,
+ * else ceil(persistent_cache_size / (block_t * block_h * block_w)); 0 in dense mode. */
 PBSA_API int pbsa_num_slots(const pbsa_config* cfg);
 /* k, local blocks attended per query block for a window of local_frames frames:
- * N_L = local_frames * NB_f; k = N_L when use_local_block_sparse_attn is 0 or in dense
+ * N_L = local_frames / block_t * NB; k = N_L when use_local_block_sparse_attn is 0 or in dense
  * mode, else clamp(ceil(ratio * N_L), 1, N_L).  When k = N_L and no scores are asked for,
  * pbsa_select_blocks writes the full ascending list without scoring. */
 PBSA_API int pbsa_topk_count(const pbsa_config* cfg, int local_frames);
@@ -141,9 +148,9 @@ PBSA_API const char* pbsa_version(void);
  *
  *   q        [B, q_frames*T_f, H, D] bf16
  *   k_local  ring [B, W*T_f, H, D] bf16; window = local_frames frames from ring_head
- *   idx      [B, H, q_frames*NB_f, idx_stride] int32 out (idx_stride >= k)
- *   cnt      [B, H, q_frames*NB_f] int32 out
- *   scores   nullable; [B, H, q_frames*NB_f, local_frames*NB_f] fp32 out
+ *   idx      [B, H, QB, idx_stride] int32 out (QB = q_frames / block_t * NB, idx_stride >= k)
+ *   cnt      [B, H, QB] int32 out
+ *   scores   nullable; [B, H, QB, N_L] fp32 out
  *   workspace >= pbsa_workspace_size(cfg, PBSA_OP_SELECT, q_frames) bytes
  */
 PBSA_API int pbsa_select_blocks(const pbsa_config* cfg, const void* q, int q_frames,
@@ -185,16 +192,17 @@ PBSA_API int pbsa_select_blocks_noalloc(const pbsa_config* cfg, const void* q, i
  * pooled key can be computed once, when its frame is appended).  The paper has no separate
  * call for this.
  *
- * pbsa_pool_keys: mean over the valid tokens of every 1x8x8 block of the n_frames frames in
- * ring slots first_slot, first_slot+1, ... (mod W) of k_local [B, W*T_f, H, D] bf16, written
- * to kbar [B, H, W*NB_f, D] fp32 at row (slot * NB_f + block) - the layout
+ * pbsa_pool_keys: mean over the valid tokens of every block of the n_frames frames in ring
+ * slots first_slot, first_slot+1, ... (mod W) of k_local [B, W*T_f, H, D] bf16, written to
+ * kbar [B, H, (W / block_t) * NB, D] fp32 at row (slot / block_t * NB + block) - the layout
  * pbsa_select_blocks_pooled reads.  Rows of other slots are left as they are.  kbar is
- * caller-owned device memory; no workspace.  PBSA_ERR_ARG on a bad slot/frame count.
+ * caller-owned device memory; no workspace.  PBSA_ERR_ARG on a bad slot/frame count
+ * (both multiples of block_t).
  *
  * pbsa_select_blocks_pooled: pbsa_select_blocks with the window's key means taken from kbar
  * (every slot of the window must have been pooled since its frame was written) instead of
  * being recomputed from k_local: only the chunk's queries are pooled.  Same outputs and
- * errors as pbsa_select_blocks; workspace >= B*H*q_frames*NB_f*D*4 bytes (256-aligned),
+ * errors as pbsa_select_blocks; workspace >= B*H*QB*D*4 bytes (256-aligned),
  * not needed when every block is selected and scores is NULL.
  */
 PBSA_API int pbsa_pool_keys(const pbsa_config* cfg, const void* k_local, int first_slot, int n_frames,
@@ -214,8 +222,8 @@ PBSA_API int pbsa_select_blocks_pooled(const pbsa_config* cfg, const void* q, in
  *
  *   out        [B, q_frames*T_f, H, D] bf16 out
  *   lse        [B, H, q_frames*T_f] fp32 out, natural-log softmax normaliser per row
- *   mass_local nullable; [B, H, W*NB_f] fp32, indexed by PHYSICAL block
- *              (ring slot * NB_f + block in frame).  Accumulated (+=): the softmax
+ *   mass_local nullable; [B, H, (W / block_t) * NB] fp32, indexed by PHYSICAL block
+ *              (ring slot / block_t * NB + block in group).  Accumulated (+=): the softmax
  *              probability summed over this chunk's query rows, per local block.
  *   mass_pers  nullable; [B, H, S] fp32, accumulated the same way per persistent slot.
  *              This is the pers_score array of pbsa_cache_update.
@@ -261,14 +269,15 @@ PBSA_API int pbsa_attn_bwd(const pbsa_config* cfg, const void* q, int q_frames,
  * mass_local of their physical block).  Ordered by score descending, ties by that
  * candidate order, the first min(S, #candidates) are kept.  Kept slots stay in place;
  * the free slots (empty ones ascending, then dropped ones ascending) receive the kept
- * evicted blocks in id order: tokens copied in raster order, pers_len = token count,
- * pers_score = the block's mass, pers_src = global frame * NB_f + block in frame, where
- * the oldest window frame has global number first_frame_global.  Dropped slots that
+ * evicted blocks in id order: tokens copied frame by frame in raster order, pers_len =
+ * token count, pers_score = the block's mass, pers_src = global frame group * NB + block
+ * in group (global frame group = global frame / block_t), where the oldest window frame
+ * has global number first_frame_global.  Dropped slots that
  * receive nothing become empty (len 0, score 0, src -1).  The evicted blocks'
  * mass_local entries are reset to 0.  The caller then advances its ring:
  * ring_head = (ring_head + n_evict_frames) % W, local_frames -= n_evict_frames.
  *
- *   upd    [B, H, n_evict_frames*NB_f, 2] int32 out: (slot, logical block id) per
+ *   upd    [B, H, n_evict_frames / block_t * NB, 2] int32 out: (slot, logical block id) per
  *          admission, in admission order
  *   n_upd  [B, H] int32 out: admissions per (b, h)
  *   workspace >= pbsa_workspace_size(cfg, PBSA_OP_UPDATE, 0) bytes

@@ -62,9 +62,10 @@ class Buffers:
         W = P.pbsa_window_frames(cfg)
         S = P.pbsa_num_slots(cfg)
         assert S == slot_count(wl)
-        self.nbf, self.W, self.S, self.tf = nbf, W, S, tf
-        self.qb = q_frames * nbf
-        self.nl = local_frames * nbf
+        bt = cfg.block_t
+        self.nbf, self.W, self.S, self.tf, self.bt = nbf, W, S, tf, bt
+        self.qb = q_frames // bt * nbf
+        self.nl = local_frames // bt * nbf
         self.k = P.pbsa_topk_count(cfg, local_frames)
         self.idx_stride = self.k if idx_stride is None else idx_stride
         B, H, D = wl.B, wl.H, wl.D
@@ -81,7 +82,7 @@ class Buffers:
                                   dtype=torch.uint8, device=dev)
         self.out = torch.full((B, q_frames * tf, H, D), float("nan"), dtype=torch.bfloat16, device=dev)
         self.lse = torch.full((B, H, q_frames * tf), float("nan"), **f32)
-        self.mass_local = torch.zeros((B, H, W * nbf), **f32)
+        self.mass_local = torch.zeros((B, H, W // bt * nbf), **f32)
         self.mass_pers = torch.zeros((B, H, S), **f32)
         self.status = torch.zeros(1, **i32)
 

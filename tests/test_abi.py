@@ -20,18 +20,39 @@ def test_library_exports_every_header_symbol():
         assert hasattr(lib, n), n
 
 
-@pytest.mark.parametrize("name", ["tiny", "decode", "rollout", "train"])
+@pytest.mark.parametrize("name", ["tiny", "decode", "rollout", "train", "decode344"])
 def test_geometry_matches_oracle(name):
     wl = WORKLOADS[name]
     cfg = config(wl)
     P.pbsa_validate_config(cfg)
-    nbf = len(orc.frame_blocks(wl.frame_h, wl.frame_w))
+    bt, bh, bw = wl.block
+    nbf = len(orc.frame_blocks(wl.frame_h, wl.frame_w, bh, bw, bt))
     assert P.pbsa_blocks_per_frame(cfg) == nbf
     assert P.pbsa_window_frames(cfg) == wl.window_frames
     assert P.pbsa_num_slots(cfg) == slot_count(wl) == orc.n_slots(
-        wl.persistent_cache_size, wl.frame_h, wl.frame_w)
-    for lf in range(1, wl.window_frames + 1):
-        assert P.pbsa_topk_count(cfg, lf) == orc.topk_count(wl.topk_ratio, lf * nbf)
+        wl.persistent_cache_size, wl.frame_h, wl.frame_w, bh, bw, bt)
+    for lf in range(bt, wl.window_frames + 1, bt):
+        assert P.pbsa_topk_count(cfg, lf) == orc.topk_count(wl.topk_ratio, lf // bt * nbf)
+
+
+def test_block344_page_sizes():
+    cfg = config(WORKLOADS["decode344"])
+    assert P.pbsa_blocks_per_frame(cfg) == 104        # 8 block rows (last 2 high) x 13
+    assert P.pbsa_num_slots(cfg) == 208
+    assert P.pbsa_topk_count(cfg, 6) == 26            # ceil(0.125 * 208)
+    assert P.pbsa_topk_count(cfg, 3) == 13
+    lib = P.library()
+    # frame counts that are not whole 3-frame groups are rejected before any launch
+    rc = lib.pbsa_select_blocks(ctypes.byref(cfg), 256, 3, 256, 4, 0, 256, 26, 256, None, 256,
+                                1 << 30, None)
+    assert rc == P.PBSA_ERR_ARG and "block_t" in P.pbsa_last_error()
+    # a 6-frame window is not a whole number of 4-frame groups
+    with pytest.raises(P.PBSAError) as e:
+        P.pbsa_validate_config(config(WORKLOADS["decode"], sparse_kv_block_size=(4, 4, 4)))
+    assert e.value.code == P.PBSA_ERR_ARG
+    rc = lib.pbsa_cache_update(ctypes.byref(cfg), 256, 256, 6, 0, 256, 2, 0, 256, 256, 256,
+                               256, 256, 256, 256, None, 0, None)
+    assert rc == P.PBSA_ERR_ARG and "block_t" in P.pbsa_last_error()
 
 
 def test_page_defaults_give_21_of_168():
@@ -50,7 +71,8 @@ def test_page_defaults_give_21_of_168():
     ("local_cache_size", 9000, P.PBSA_ERR_ARG),
     ("local_block_sparse_topk_ratio", 0.0, P.PBSA_ERR_ARG),
     ("local_block_sparse_topk_ratio", 1.5, P.PBSA_ERR_ARG),
-    ("block_h", 4, P.PBSA_ERR_UNSUPPORTED),
+    ("block_h", 9, P.PBSA_ERR_UNSUPPORTED),      # 1 x 9 x 8 = 72 tokens > 64
+    ("block_t", 0, P.PBSA_ERR_ARG),
     ("kv_cache_mode", 3, P.PBSA_ERR_UNSUPPORTED),
     ("max_seq_len", 100, P.PBSA_ERR_ARG),
     ("B", 0, P.PBSA_ERR_ARG),

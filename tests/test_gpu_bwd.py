@@ -76,9 +76,10 @@ def _run_case(wl, dev, ring_head=0, local_frames=None, persistent_filled=True, c
     kwin = ring_to_window(kring.cpu(), ring_head, lf, W, tf)
     vwin = ring_to_window(vring.cpu(), ring_head, lf, W, tf)
     idx = buf.idx.cpu().numpy()[..., :buf.k]
+    bt, bh, bw = wl.block
     want = orc.attn_bwd(f64(inp["q"]), f64(inp["k_pers"]), f64(inp["v_pers"]),
                         inp["pers_len"].numpy(), f64(kwin), f64(vwin), idx, f64(dout),
-                        wl.frame_h, wl.frame_w)
+                        wl.frame_h, wl.frame_w, bh, bw, bt=bt)
     return _check_grads(g, want, inp["pers_len"], ring_head, lf, W, tf, wl.name)
 
 

@@ -19,10 +19,11 @@ from tests.harness import (LSE_ABS, MASS_ABS, MASS_REL, assert_close_bf16, check
 pytestmark = pytest.mark.gpu
 
 
-def _logical_mass(ml_phys, ring_head, local_frames, W, nbf):
-    out = np.zeros(ml_phys.shape[:2] + (local_frames * nbf,))
-    for lid in range(local_frames * nbf):
-        out[:, :, lid] = ml_phys[:, :, ((ring_head + lid // nbf) % W) * nbf + lid % nbf]
+def _logical_mass(ml_phys, ring_head, local_frames, W, nbf, bt=1):
+    Wg = W // bt
+    out = np.zeros(ml_phys.shape[:2] + (local_frames // bt * nbf,))
+    for lid in range(local_frames // bt * nbf):
+        out[:, :, lid] = ml_phys[:, :, ((ring_head // bt + lid // nbf) % Wg) * nbf + lid % nbf]
     return out
 
 
@@ -34,7 +35,7 @@ def _state_from_gpu(a, W, tf, nbf):
                      np.zeros((t.shape[0], 0) + tuple(t.shape[2:])))
     return orc.DecodeState(
         win(a.k_local), win(a.v_local),
-        _logical_mass(a.mass_local.cpu().double().numpy(), rh, lf, W, nbf),
+        _logical_mass(a.mass_local.cpu().double().numpy(), rh, lf, W, nbf, a.bt),
         f64(a.k_pers), f64(a.v_pers), a.pers_len.cpu().numpy(),
         a.pers_score.cpu().double().numpy(), a.pers_src.cpu().numpy(), a.first_frame_global)
 
@@ -42,10 +43,11 @@ def _state_from_gpu(a, W, tf, nbf):
 def _run_rollout(wl, dev, chunks, chunk_fn):
     a = SparseForcingAttention(wl.B, wl.H, wl.D, wl.frame_h, wl.frame_w, wl.total_cache_size,
                                wl.local_cache_size, wl.persistent_cache_size,
-                               max_seq_len=wl.max_seq_len,
+                               sparse_kv_block_size=wl.block, max_seq_len=wl.max_seq_len,
                                local_block_sparse_topk_ratio=wl.topk_ratio,
                                chunk_frames=wl.q_frames, device=dev)
     W, tf, nbf, S = a.W, a.tf, a.nbf, a.S
+    bt, bh, bw = wl.block
     exact_frac, admitted = [], []
     for step in range(chunks):
         q, k, v = chunk_fn(step)
@@ -59,16 +61,16 @@ def _run_rollout(wl, dev, chunks, chunk_fn):
         # ---- the oracle's step on the same state, with the GPU's selection (near-ties may
         # legitimately differ; the selection itself is checked against the oracle's scores)
         st1, o = orc.decode_step(st0, f64(q), f64(k), f64(v), wl.topk_ratio, W, wl.frame_h,
-                                 wl.frame_w, idx=idx[..., :P_k(a, lf)])
+                                 wl.frame_w, idx=idx[..., :P_k(a, lf)], bh=bh, bw=bw, bt=bt)
         kwin = np.concatenate([st0.win_k, f64(k)], 1)
         vwin = np.concatenate([st0.win_v, f64(v)], 1)
-        _, sc_o = orc.select_blocks(f64(q), kwin, wl.frame_h, wl.frame_w, wl.topk_ratio)
+        _, sc_o = orc.select_blocks(f64(q), kwin, wl.frame_h, wl.frame_w, wl.topk_ratio, bh=bh, bw=bw, bt=bt)
         kk = P_k(a, lf)
         exact_frac.append(check_topk(idx[..., :kk], a.cnt.cpu().numpy(), sc_o, kk))
         assert_close_bf16(f64(a.out), o["O"], f"step {step} out")
         assert np.abs(a.lse.cpu().numpy() - o["lse"]).max() <= LSE_ABS
         ps1 = a.pers_score.cpu().double().numpy()
-        ml1 = _logical_mass(a.mass_local.cpu().double().numpy(), rh, lf, W, nbf)
+        ml1 = _logical_mass(a.mass_local.cpu().double().numpy(), rh, lf, W, nbf, bt)
         assert np.allclose(ps1, o["pers_score_before_merge"], rtol=MASS_REL, atol=MASS_ABS)
         assert np.allclose(ml1, o["win_mass_before_merge"], rtol=MASS_REL, atol=MASS_ABS)
         # ---- slide + merge: the eviction count is the oracle's
@@ -80,7 +82,8 @@ def _run_rollout(wl, dev, chunks, chunk_fn):
             ups = [tuple(x) for x in a.upd[0, 0, :nup[0]].cpu().numpy()]
             # decisions on the GPU's own masses must match the oracle's merge exactly
             r = orc.cache_update(st0.k_pers, st0.v_pers, st0.pers_len, ps1, st0.pers_src, kwin,
-                                 vwin, ml1, n_ev, st0.first_frame_global, wl.frame_h, wl.frame_w)
+                                 vwin, ml1, n_ev, st0.first_frame_global, wl.frame_h, wl.frame_w,
+                                 bh, bw, bt)
             assert ups == r["updates"][0][0], f"step {step}"
             assert np.array_equal(a.pers_len.cpu().numpy(), r["pers_len"])
             assert np.array_equal(a.pers_src.cpu().numpy(), r["pers_src"])
@@ -89,7 +92,7 @@ def _run_rollout(wl, dev, chunks, chunk_fn):
             # and the oracle's own step (its masses) decides the same wherever the keep/drop
             # margin exceeds 1e-3
             cand = [o["pers_score_before_merge"][0, 0, s] for s in range(S) if st0.pers_len[0, 0, s] > 0]
-            cand += list(o["win_mass_before_merge"][0, 0, :n_ev * nbf])
+            cand += list(o["win_mass_before_merge"][0, 0, :n_ev // bt * nbf])
             srt = sorted(cand, reverse=True)
             margin = (srt[S - 1] - srt[S]) if len(srt) > S else np.inf
             if margin > 1e-3:

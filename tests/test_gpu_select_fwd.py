@@ -27,11 +27,13 @@ ODDQB = Workload("oddqb", B=1, H=3, D=128, frame_h=16, frame_w=24,
                  max_seq_len=8 * 384, q_frames=1, topk_ratio=0.5, seed=7)
 
 
-def _mass_to_phys(ml_logical, ring_head, local_frames, W, nbf):
+def _mass_to_phys(ml_logical, ring_head, local_frames, W, nbf, bt=1):
+    """Masses by logical block -> by physical block (ring frame group * NB + block)."""
     B, H, _ = ml_logical.shape
-    out = np.zeros((B, H, W * nbf))
-    for lid in range(local_frames * nbf):
-        phys = ((ring_head + lid // nbf) % W) * nbf + lid % nbf
+    Wg = W // bt
+    out = np.zeros((B, H, Wg * nbf))
+    for lid in range(local_frames // bt * nbf):
+        phys = ((ring_head // bt + lid // nbf) % Wg) * nbf + lid % nbf
         out[:, :, phys] = ml_logical[:, :, lid]
     return out
 
@@ -59,8 +61,10 @@ def _run_case(wl, dev, ring_head=0, local_frames=None, persistent_filled=True, c
     # --- selection
     kwin = ring_to_window(kring.cpu(), ring_head, lf, W, tf)
     vwin = ring_to_window(vring.cpu(), ring_head, lf, W, tf)
+    bt, bh, bw = wl.block
     idx_o, sc_o = orc.select_blocks(f64(inp["q"]), f64(kwin), wl.frame_h, wl.frame_w,
-                                    wl.topk_ratio, use_sparse=bool(cfg.use_local_block_sparse_attn))
+                                    wl.topk_ratio, use_sparse=bool(cfg.use_local_block_sparse_attn),
+                                    bh=bh, bw=bw, bt=bt)
     k = buf.k
     assert idx_o.shape[-1] == k
     assert np.allclose(buf.scores.cpu().numpy(), sc_o, rtol=0, atol=1e-5)
@@ -70,7 +74,7 @@ def _run_case(wl, dev, ring_head=0, local_frames=None, persistent_filled=True, c
     # --- forward, on the GPU's selection
     O, lse, mp, ml = orc.attn_fwd(f64(inp["q"]), f64(inp["k_pers"]), f64(inp["v_pers"]),
                                   inp["pers_len"].numpy(), f64(kwin), f64(vwin), idx_g[..., :k],
-                                  wl.frame_h, wl.frame_w, heads=heads, qblocks=qblocks)
+                                  wl.frame_h, wl.frame_w, bh, bw, heads=heads, qblocks=qblocks, bt=bt)
     out = f64(buf.out)
     lse_g = buf.lse.cpu().numpy()
     sel = ~np.isnan(lse)
@@ -91,7 +95,7 @@ def _run_case(wl, dev, ring_head=0, local_frames=None, persistent_filled=True, c
         tot = mlg.sum(-1) + mpg.sum(-1)
         assert np.allclose(tot, wl.nq, rtol=1e-4), tot
         if heads is None and qblocks is None:
-            want_l = _mass_to_phys(ml, ring_head, lf, W, buf.nbf)
+            want_l = _mass_to_phys(ml, ring_head, lf, W, buf.nbf, bt)
             assert np.allclose(mlg, want_l, rtol=MASS_REL, atol=MASS_ABS)
             assert np.allclose(mpg, mp, rtol=MASS_REL, atol=MASS_ABS)
     return frac
