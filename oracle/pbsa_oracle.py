@@ -40,7 +40,8 @@ import numpy as np
 
 __all__ = ["frame_blocks", "topk_count", "pool_blocks", "block_scores", "select_topk",
            "select_blocks", "attend_rows", "attn_fwd", "cache_update", "attn_bwd",
-           "slot_capacity", "n_slots", "evict_count", "DecodeState", "decode_step"]
+           "slot_capacity", "n_slots", "sink_slots", "evict_count", "append_frames",
+           "DecodeState", "decode_step"]
 
 
 # ---------------------------------------------------------------------------------------
@@ -82,6 +83,17 @@ def n_slots(persistent_cache_size: int, frame_h: int, frame_w: int, bh=8, bw=8, 
     if persistent_cache_size % tg == 0:
         return persistent_cache_size // tg * len(frame_blocks(frame_h, frame_w, bh, bw, bt))
     return -(-persistent_cache_size // (bt * bh * bw))
+
+
+def sink_slots(sink_frames: int, frame_h: int, frame_w: int, bh=8, bw=8, bt=1) -> int:
+    """Persistent slots reserved for the sink (project page, kernel features: "local, sink,
+    and learned top-k" sparsity patterns).  Reading: the sink is the first sink_frames
+    frames of the sequence (a multiple of bt); each of their blocks keeps one slot of its
+    own at the front of the slot store, in addition to the slots of persistent_cache_size,
+    so that every query attends to them for the whole sequence."""
+    if sink_frames % bt:
+        raise ValueError("sink_frames must be a multiple of the block's frame count")
+    return sink_frames // bt * len(frame_blocks(frame_h, frame_w, bh, bw, bt))
 
 
 def cache_geometry(kv_cache_mode: str, total_cache_size: int, local_cache_size: int,
@@ -271,7 +283,8 @@ def attn_fwd(q, k_pers, v_pers, pers_len, k_win, v_win, idx, frame_h, frame_w,
 # algorithm fragment: the t=0 pass updates P and L)
 # ---------------------------------------------------------------------------------------
 def cache_update(k_pers, v_pers, pers_len, pers_score, pers_src, k_win, v_win, mass_local,
-                 n_evict_frames, first_frame_global, frame_h, frame_w, bh=8, bw=8, bt=1):
+                 n_evict_frames, first_frame_global, frame_h, frame_w, bh=8, bw=8, bt=1,
+                 n_sink=0):
     """Slide the window by n_evict_frames and merge the evicted blocks into the
     persistent set by accumulated attention mass.
 
@@ -292,7 +305,8 @@ def cache_update(k_pers, v_pers, pers_len, pers_score, pers_src, k_win, v_win, m
       (global frame group * NB + block in group, the group of global frames
       bt*g .. bt*g + bt - 1 being number g) as source.  Dropped slots not refilled end
       empty (length 0, score 0, source -1).  n_evict_frames and first_frame_global are
-      multiples of bt.
+      multiples of bt.  The first n_sink slots hold sink blocks (sink_slots): they are
+      neither candidates nor free slots, and S counts only the slots after them.
 
     Returns dict(k_pers, v_pers, pers_len, pers_score, pers_src, updates) where updates
     [b][h] is the list of (slot, logical block id) admissions in admission order.
@@ -307,18 +321,20 @@ def cache_update(k_pers, v_pers, pers_len, pers_score, pers_src, k_win, v_win, m
     plen = np.array(pers_len, dtype=np.int64)
     pscore = np.array(pers_score, dtype=np.float64)
     psrc = np.array(pers_src, dtype=np.int64)
-    B, H, S = plen.shape
+    B, H, S_all = plen.shape
+    S = S_all - n_sink                  # slots that take part in the merge
     n_ev = n_evict_frames // bt * nbf
     updates = [[None] * H for _ in range(B)]
     for b in range(B):
         for h in range(H):
-            occupied = [s for s in range(S) if plen[b, h, s] > 0]
+            mergeable = range(n_sink, S_all)
+            occupied = [s for s in mergeable if plen[b, h, s] > 0]
             cands = [("slot", s, float(pscore[b, h, s])) for s in occupied]
             cands += [("block", j, float(mass_local[b, h, j])) for j in range(n_ev)]
             order = sorted(range(len(cands)), key=lambda c: (-cands[c][2], c))
             kept = set(order[:min(S, len(cands))])
             dropped = [cands[c][1] for c in range(len(occupied)) if c not in kept]
-            free = [s for s in range(S) if plen[b, h, s] == 0] + sorted(dropped)
+            free = [s for s in mergeable if plen[b, h, s] == 0] + sorted(dropped)
             for s in dropped:
                 plen[b, h, s] = 0
                 pscore[b, h, s] = 0.0
@@ -418,6 +434,52 @@ def evict_count(frames_in_window: int, chunk_frames: int, window_frames: int) ->
     return max(0, frames_in_window + chunk_frames - window_frames)
 
 
+def append_frames(state, k_new, v_new, sink_frames, frame_h, frame_w, bh=8, bw=8, bt=1):
+    """New frames join the cache (algorithm fragment: each chunk's frames enter the KV
+    cache).  The first frame appended has global number first_frame_global + the window's
+    frame count.  Frames whose global number is below sink_frames are sink frames
+    (sink_slots): each of their blocks is written, whole, into its reserved slot
+    (slot = global frame group * NB + block in group), with its token count as length,
+    score 0 and its global id as source, and they do not enter the window; sink frames
+    come first in a sequence, so the window is still empty then and its oldest frame
+    becomes the first frame after them.  Every other frame joins the window after its
+    newest frame.  Returns the new state; the input is not modified."""
+    blocks = frame_blocks(frame_h, frame_w, bh, bw, bt)
+    nbf = len(blocks)
+    tf = frame_h * frame_w
+    k_new = np.asarray(k_new, np.float64)
+    v_new = np.asarray(v_new, np.float64)
+    n = k_new.shape[1] // tf
+    win_frames = state.win_k.shape[1] // tf
+    g0 = state.first_frame_global + win_frames
+    if g0 % bt or n % bt:
+        raise ValueError("frames are appended in whole frame groups")
+    n_sink_new = max(0, min(n, sink_frames - g0))
+    if n_sink_new and win_frames:
+        raise ValueError("sink frames come before every window frame")
+    kp, vp = state.k_pers.copy(), state.v_pers.copy()
+    plen, pscore, psrc = state.pers_len.copy(), state.pers_score.copy(), state.pers_src.copy()
+    B, H = plen.shape[:2]
+    for f in range(0, n_sink_new, bt):                       # one frame group at a time
+        grp = (g0 + f) // bt
+        for i, toks in enumerate(blocks):
+            s = grp * nbf + i
+            kp[:, :, s] = 0.0
+            vp[:, :, s] = 0.0
+            for b in range(B):
+                for h in range(H):
+                    kp[b, h, s, :len(toks)] = k_new[b, f * tf + toks, h, :]
+                    vp[b, h, s, :len(toks)] = v_new[b, f * tf + toks, h, :]
+            plen[:, :, s] = len(toks)
+            pscore[:, :, s] = 0.0
+            psrc[:, :, s] = s
+    rest = slice(n_sink_new * tf, n * tf)
+    return DecodeState(np.concatenate([state.win_k, k_new[:, rest]], 1),
+                       np.concatenate([state.win_v, v_new[:, rest]], 1),
+                       np.concatenate([state.win_mass, np.zeros((B, H, (n - n_sink_new) // bt * nbf))], 2),
+                       kp, vp, plen, pscore, psrc, state.first_frame_global + n_sink_new)
+
+
 class DecodeState:
     """Cache state between chunks, in the oracle's own plain layout (one batch item list
     entry per array axis as in the other oracle functions):
@@ -450,11 +512,11 @@ class DecodeState:
 
 
 def decode_step(state: DecodeState, q, k_chunk, v_chunk, ratio, window_frames, frame_h,
-                frame_w, use_sparse=True, idx=None, bh=8, bw=8, bt=1):
+                frame_w, use_sparse=True, idx=None, bh=8, bw=8, bt=1, sink_frames=0):
     """One chunk's cache pass, in the order of the algorithm fragment:
 
-      1. the chunk's frames join the window (reading: before its attention, so the window
-         includes the current chunk);
+      1. the chunk's frames join the cache (append_frames; reading: before its attention,
+         so the window includes the current chunk; sink frames go to their slots);
       2. top-k block selection over the window (select_blocks), unless `idx` is given
          (a caller may pass another implementation's selection to compare the rest of the
          step on equal terms);
@@ -463,7 +525,8 @@ def decode_step(state: DecodeState, q, k_chunk, v_chunk, ratio, window_frames, f
          probability mass it received in this pass (reading: per head, never decayed);
       5. slide: evict_count(frames, chunk frames, window_frames) oldest frames leave the
          window, and their blocks are merged into the persistent cache by accumulated mass
-         (cache_update); the evicted blocks' masses leave with them.
+         (cache_update, the sink slots taking no part); the evicted blocks' masses leave
+         with them.
 
     Returns (new_state, out) with out = dict(idx, scores, O, lse, mass_pers, mass_local,
     n_evict, updates).  The input state is not modified.
@@ -471,33 +534,35 @@ def decode_step(state: DecodeState, q, k_chunk, v_chunk, ratio, window_frames, f
     nbf = len(frame_blocks(frame_h, frame_w, bh, bw, bt))
     tf = frame_h * frame_w
     chunk_frames = np.asarray(k_chunk).shape[1] // tf
-    frames = state.win_k.shape[1] // tf + chunk_frames
+    n_sink = sink_slots(sink_frames, frame_h, frame_w, bh, bw, bt)
+    appended = append_frames(state, k_chunk, v_chunk, sink_frames, frame_h, frame_w, bh, bw, bt)
+    frames = appended.win_k.shape[1] // tf
     if frames > window_frames:
         raise ValueError("the window has no room for the chunk")
-    win_k = np.concatenate([state.win_k, np.asarray(k_chunk, np.float64)], axis=1)
-    win_v = np.concatenate([state.win_v, np.asarray(v_chunk, np.float64)], axis=1)
+    win_k, win_v, win_mass = appended.win_k, appended.win_v, appended.win_mass
     B, H = state.pers_len.shape[:2]
-    win_mass = np.concatenate([state.win_mass, np.zeros((B, H, chunk_frames // bt * nbf))], axis=2)
     scores = None
     if idx is None:
         idx, scores = select_blocks(q, win_k, frame_h, frame_w, ratio, use_sparse, bh, bw, bt)
-    O, lse, mass_pers, mass_local = attn_fwd(q, state.k_pers, state.v_pers, state.pers_len,
-                                             win_k, win_v, idx, frame_h, frame_w, bh, bw, bt=bt)
+    O, lse, mass_pers, mass_local = attn_fwd(q, appended.k_pers, appended.v_pers,
+                                             appended.pers_len, win_k, win_v, idx, frame_h,
+                                             frame_w, bh, bw, bt=bt)
     win_mass = win_mass + mass_local
-    pers_score = state.pers_score + mass_pers
+    pers_score = appended.pers_score + mass_pers
     n_ev = evict_count(frames, chunk_frames, window_frames)
     out = dict(idx=idx, scores=scores, O=O, lse=lse, mass_pers=mass_pers,
                mass_local=mass_local, n_evict=n_ev, updates=[[[] for _ in range(H)] for _ in range(B)],
                pers_score_before_merge=pers_score, win_mass_before_merge=win_mass)
     if n_ev == 0:
-        new = DecodeState(win_k, win_v, win_mass, state.k_pers, state.v_pers, state.pers_len,
-                          pers_score, state.pers_src, state.first_frame_global)
+        new = DecodeState(win_k, win_v, win_mass, appended.k_pers, appended.v_pers,
+                          appended.pers_len, pers_score, appended.pers_src,
+                          appended.first_frame_global)
         return new, out
-    r = cache_update(state.k_pers, state.v_pers, state.pers_len, pers_score, state.pers_src,
-                     win_k, win_v, win_mass, n_ev, state.first_frame_global, frame_h, frame_w,
-                     bh, bw, bt)
+    r = cache_update(appended.k_pers, appended.v_pers, appended.pers_len, pers_score,
+                     appended.pers_src, win_k, win_v, win_mass, n_ev,
+                     appended.first_frame_global, frame_h, frame_w, bh, bw, bt, n_sink)
     out["updates"] = r["updates"]
     new = DecodeState(win_k[:, n_ev * tf:], win_v[:, n_ev * tf:], win_mass[:, :, n_ev // bt * nbf:],
                       r["k_pers"], r["v_pers"], r["pers_len"], r["pers_score"], r["pers_src"],
-                      state.first_frame_global + n_ev)
+                      appended.first_frame_global + n_ev)
     return new, out

@@ -709,3 +709,85 @@ def test_merge_344_hand_example():
     with pytest.raises(ValueError):
         orc.cache_update(kp, kp, plen, np.zeros((1, 1, 2)), np.zeros((1, 1, 2), int), kw, kw, ml,
                          2, 6, fh, fw, 4, 4, bt=3)
+
+
+# ------------------------------------------------------------------------------ sink
+def test_sink_slot_counts():
+    assert orc.sink_slots(1, 30, 52) == 28
+    assert orc.sink_slots(2, 16, 16) == 8
+    assert orc.sink_slots(3, 30, 52, 4, 4, 3) == 104
+    assert orc.sink_slots(0, 30, 52) == 0
+    with pytest.raises(ValueError):
+        orc.sink_slots(2, 30, 52, 4, 4, 3)
+
+
+def test_merge_never_touches_sink_slots():
+    # Without a sink, the candidates 0.01, 5, 1 (slots) and 3, 0.5 (blocks) keep slot 1,
+    # block 0 and slot 2: slot 0 is dropped and receives block 0.
+    r, _, _ = _merge_case(3, [64, 64, 32], [0.01, 5.0, 1.0], [3.0, 0.5])
+    assert r["updates"][0][0] == [(0, 0)]
+    # With slot 0 a sink slot, 2 ordinary slots compete: 5, 1, 3, 0.5 keep slot 1 and
+    # block 0; slot 2 is dropped and receives block 0.  The sink slot stays although every
+    # candidate beats it.
+    fh, fw, D = 8, 12, 2
+    kp = np.zeros((1, 1, 3, 64, D))
+    kp[0, 0, 0, :64] = 7.0
+    plen = np.array([[[64, 64, 32]]])
+    kw = np.arange(2 * 96 * D, dtype=np.float64).reshape(1, 2 * 96, 1, D)
+    ml = np.zeros((1, 1, 4))
+    ml[0, 0, :2] = [3.0, 0.5]
+    r = orc.cache_update(kp, kp, plen, np.array([[[0.01, 5.0, 1.0]]]), np.array([[[0, 11, 12]]]),
+                         kw, kw, ml, 1, 2, fh, fw, n_sink=1)
+    assert r["updates"][0][0] == [(2, 0)]
+    assert r["pers_src"].tolist() == [[[0, 11, 2 * 2 + 0]]]
+    assert r["pers_score"].tolist() == [[[0.01, 5.0, 3.0]]]
+    assert (r["k_pers"][0, 0, 0, :64] == 7.0).all()
+
+
+def test_decode_step_with_a_sink_frame_hand_rollout():
+    """Frames of 8x8 tokens (one block), D = 4, 2-frame chunks, a 4-frame window, 2 ordinary
+    slots and a 1-frame sink, ratio 1 (every window block).  Queries are (2, 0, 0, 0); the
+    sink frame's keys are (-10, 0, 0, 0) (logit -10), every other key is zero (logit 0)."""
+    fh = fw = 8
+    D, tf = 4, 64
+    rng = np.random.default_rng(4)
+    chunks = []
+    for c in range(3):
+        q = np.zeros((1, 2 * tf, 1, D))
+        q[..., 0] = 2.0
+        k = np.zeros((1, 2 * tf, 1, D))
+        if c == 0:
+            k[0, :tf, 0, 0] = -10.0          # global frame 0: the sink
+        chunks.append((q, k, rng.standard_normal((1, 2 * tf, 1, D))))
+    n_sink = orc.sink_slots(1, fh, fw)
+    st = orc.DecodeState.empty(1, 1, D, n_sink + 2, fh, fw)
+    res = []
+    for q, k, v in chunks:
+        st, o = orc.decode_step(st, q, k, v, 1.0, 4, fh, fw, sink_frames=1)
+        res.append((st, o))
+    e = math.exp(-10.0)
+    # chunk 0: frame 0 goes to sink slot 0, frame 1 into the window; 128 query rows over
+    # 64 sink keys (weight e^-10) and 64 window keys (weight 1)
+    st0, o0 = res[0]
+    assert st0.win_k.shape[1] == tf and st0.first_frame_global == 1 and o0["n_evict"] == 0
+    assert st0.pers_len.tolist() == [[[64, 0, 0]]] and st0.pers_src.tolist() == [[[0, -1, -1]]]
+    assert np.allclose(o0["mass_pers"][0, 0, 0], 128 * e / (1 + e), rtol=1e-12)
+    assert np.allclose(o0["mass_local"][0, 0], [128 / (1 + e)], rtol=1e-12)
+    # chunk 1: window [f1, f2, f3]; Z = 64 e + 192; then f1 leaves and takes ordinary slot 1
+    Z1 = 64 * e + 192
+    st1, o1 = res[1]
+    assert np.allclose(o1["mass_local"][0, 0], [8192 / Z1] * 3, rtol=1e-12)
+    assert o1["n_evict"] == 1 and o1["updates"][0][0] == [(1, 0)]
+    assert st1.pers_src.tolist() == [[[0, 1, -1]]]
+    assert np.allclose(st1.pers_score[0, 0, 1], 128 / (1 + e) + 8192 / Z1, rtol=1e-12)
+    # chunk 2: window [f2 .. f5]; Z = 64 e + 320; f2 and f3 leave with equal masses; the one
+    # free ordinary slot goes to f2 (the lower id) and f3 is dropped; the sink slot, whose
+    # mass is the smallest of all, is no candidate and stays
+    Z2 = 64 * e + 320
+    st2, o2 = res[2]
+    assert o2["n_evict"] == 2 and o2["updates"][0][0] == [(2, 0)]
+    assert st2.pers_src.tolist() == [[[0, 1, 2]]] and st2.pers_len.tolist() == [[[64, 64, 64]]]
+    assert np.allclose(st2.pers_score[0, 0, 2], 8192 / Z1 + 8192 / Z2, rtol=1e-12)
+    assert st2.pers_score[0, 0, 0] < 1e-2 < st2.pers_score[0, 0, 2]
+    assert (st2.k_pers[0, 0, 0, :, 0] == -10.0).all()
+    assert st2.first_frame_global == 4 and st2.win_k.shape[1] == 2 * tf
