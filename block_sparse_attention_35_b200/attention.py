@@ -8,7 +8,8 @@ Every step of the method runs in the CUDA kernels behind ``pbsa.pbsa_*``.
 Typical t=0 decode pass for one chunk (pith.science page, algorithm fragment: the KV pass
 applies PBSA with top-k and updates P and L):
 
-    attn.append(k_chunk, v_chunk)        # new frames enter the ring (the window)
+    attn.append(k_chunk, v_chunk)        # new frames enter the ring (the window), their key
+                                         # means the key-mean cache; sink frames their slots
     out = attn(q_chunk, accumulate_mass=True)   # select + forward (+ block mass)
     attn.slide()                         # evict old frames, merge them into P
 """
@@ -26,13 +27,15 @@ class SparseForcingAttention:
                  sparse_kv_block_size=(1, 8, 8), max_seq_len: int = 32760,
                  use_local_block_sparse_attn: bool = True,
                  local_block_sparse_topk_ratio: float = 0.125, chunk_frames: int = 3,
-                 device="cuda"):
+                 sink_frames: int = 0, device="cuda"):
         # kv_cache_mode="dense": one window of total_cache_size tokens, no persistent slots
-        # (S = 0), every block attended; slide() then only drops the oldest frames
+        # (S = 0), every block attended; slide() then only drops the oldest frames.
+        # sink_frames: the first frames of the sequence are kept in sink slots, attended by
+        # every query and never evicted.
         self.cfg = P.make_config(B, H, D, frame_h, frame_w, total_cache_size, local_cache_size,
                                  persistent_cache_size, max_seq_len,
                                  local_block_sparse_topk_ratio, use_local_block_sparse_attn,
-                                 sparse_kv_block_size, kv_cache_mode)
+                                 sparse_kv_block_size, kv_cache_mode, sink_frames)
         P.pbsa_validate_config(self.cfg)
         self.B, self.H, self.D = B, H, D
         self.tf = frame_h * frame_w
@@ -40,6 +43,7 @@ class SparseForcingAttention:
         self.nbf = P.pbsa_blocks_per_frame(self.cfg)  # blocks per frame group
         self.W = P.pbsa_window_frames(self.cfg)
         self.S = P.pbsa_num_slots(self.cfg)
+        self.n_sink = P.pbsa_sink_slots(self.cfg)
         if chunk_frames % self.bt:
             raise ValueError("chunk_frames must be a multiple of the block's frame count")
         self.chunk_frames = chunk_frames
@@ -58,9 +62,11 @@ class SparseForcingAttention:
         self.pers_score = torch.zeros(B, H, self.S, **f32)
         self.pers_src = torch.full((B, H, self.S), -1, **i32)
         self.mass_local = torch.zeros(B, H, self.W // self.bt * self.nbf, **f32)
+        self.kbar = torch.zeros(B, H, self.W // self.bt * self.nbf, D, **f32)   # key means by ring slot
         self.ring_head = 0
         self.local_frames = 0
-        self.first_frame_global = 0
+        self.first_frame_global = 0   # global number of the oldest window frame
+        self.frames_seen = 0          # frames appended so far (sink frames included)
         # per-chunk buffers
         qf = chunk_frames
         qb = qf // self.bt * self.nbf
@@ -89,17 +95,32 @@ class SparseForcingAttention:
         return t[:, s * self.tf:(s + 1) * self.tf]
 
     def append(self, k_chunk: torch.Tensor, v_chunk: torch.Tensor):
-        """Writes the chunk's frames after the newest window frame (the window must have
-        room: call slide() first when it is full).  Accepts host (pinned) or device
-        tensors of shape [B, frames*T_f, H, D]."""
+        """The chunk's frames join the cache (the window must have room: call slide() first
+        when it is full): sink frames go to their slots, the others after the newest window
+        frame, their key means into the key-mean cache, all in one kernel.  Accepts device
+        tensors, or host (pinned) tensors that are first copied to the device, of shape
+        [B, frames*T_f, H, D] bf16."""
         n = k_chunk.shape[1] // self.tf
-        if self.local_frames + n > self.W:
+        n_sink = max(0, min(n, self.cfg.sink_frames - self.frames_seen))
+        if self.local_frames + n - n_sink > self.W:
             raise ValueError("window full: slide() before append()")
-        for f in range(n):
-            p = self.local_frames + f
-            self.frame_view(p, "k").copy_(k_chunk[:, f * self.tf:(f + 1) * self.tf], non_blocking=True)
-            self.frame_view(p, "v").copy_(v_chunk[:, f * self.tf:(f + 1) * self.tf], non_blocking=True)
-        self.local_frames += n
+        if k_chunk.device != self.device:
+            k_chunk = k_chunk.to(self.device, non_blocking=True)
+            v_chunk = v_chunk.to(self.device, non_blocking=True)
+        P.pbsa_append_frames(self.cfg, k_chunk.contiguous(), v_chunk.contiguous(), n,
+                             self.frames_seen, self.k_local, self.v_local,
+                             (self.ring_head + self.local_frames) % self.W, self.kbar,
+                             self.k_pers, self.v_pers, self.pers_len, self.pers_score,
+                             self.pers_src)
+        self.frames_seen += n
+        self.local_frames += n - n_sink
+        self.first_frame_global = self.frames_seen - self.local_frames
+
+    def pool_window(self):
+        """Recomputes the key-mean cache for every window frame, for callers that wrote the
+        ring directly instead of through append()."""
+        if self.local_frames:
+            P.pbsa_pool_keys(self.cfg, self.k_local, self.ring_head, self.local_frames, self.kbar)
 
     def load_persistent(self, k_pers, v_pers, pers_len, pers_score=None, pers_src=None):
         self.k_pers.copy_(k_pers)
@@ -112,9 +133,10 @@ class SparseForcingAttention:
 
     # ------------------------------------------------------------------ the method
     def select(self, q: torch.Tensor, q_frames: int | None = None):
+        """Top-k local blocks for the chunk, scored against the key-mean cache."""
         qf = self.chunk_frames if q_frames is None else q_frames
-        P.pbsa_select_blocks(self.cfg, q, qf, self.k_local, self.local_frames, self.ring_head,
-                             self.idx, self.kmax, self.cnt, None, self.ws_select)
+        P.pbsa_select_blocks_pooled(self.cfg, q, qf, self.kbar, self.local_frames, self.ring_head,
+                                    self.idx, self.kmax, self.cnt, None, self.ws_select)
 
     def attend(self, q: torch.Tensor, accumulate_mass: bool = False, q_frames: int | None = None):
         qf = self.chunk_frames if q_frames is None else q_frames

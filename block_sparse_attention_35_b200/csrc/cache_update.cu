@@ -3,7 +3,9 @@
 // Sparse Forcing (pith.science abstract): the persistent blocks are compressed, preserved
 // and updated; the algorithm fragment on the same page updates P and L in the t=0 pass.
 // When the oldest frames leave the local window, their blocks compete with the occupied
-// persistent slots on accumulated attention mass; the best min(S, #candidates) stay.
+// persistent slots on accumulated attention mass; the best min(S, #candidates) stay.  The
+// sink slots at the front of the store (project page: the "sink" sparsity pattern) take
+// no part: they are never candidates and never free.
 //
 // Two kernels:
 //  1. merge_rank_kernel, one CTA per (head, batch): candidates (occupied slots in slot
@@ -57,8 +59,9 @@ __global__ void __launch_bounds__(kMergeThreads) merge_rank_kernel(MergeParams p
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (warp == 0) {
         // occupied slots -> candidates 0..n_occ-1; empty slots -> head of the free list
+        // (the sink slots 0 .. n_sink-1 are neither)
         int occ = 0, emp = 0;
-        for (int s0 = 0; s0 < S; s0 += 32) {
+        for (int s0 = g.n_sink; s0 < S; s0 += 32) {
             const int s = s0 + lane;
             const bool valid = s < S;
             const bool o = valid && len[s] > 0;
@@ -94,7 +97,7 @@ __global__ void __launch_bounds__(kMergeThreads) merge_rank_kernel(MergeParams p
         const float s = sc[c];
         int rank = 0;
         for (int o = 0; o < ncand; ++o) rank += (sc[o] > s) || (sc[o] == s && o < c);
-        kept[c] = rank < S;
+        kept[c] = rank < S - g.n_sink;
     }
     __syncthreads();
     if (warp == 0) {

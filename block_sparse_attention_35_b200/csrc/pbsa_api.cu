@@ -46,12 +46,18 @@ bool dense_mode(const pbsa_config* c) { return c->kv_cache_mode == PBSA_KV_CACHE
 // tokens of the local ring: the local cache, or the whole cache in dense mode
 int window_tokens(const pbsa_config* c) { return dense_mode(c) ? c->total_cache_size : c->local_cache_size; }
 
+int sink_slot_count(const pbsa_config* c) {
+    return dense_mode(c) ? 0 : c->sink_frames / c->block_t * blocks_per_frame(c);
+}
+
+// sink slots, then the slots of persistent_cache_size
 int num_slots(const pbsa_config* c) {
     if (dense_mode(c)) return 0;
+    const int n_sink = sink_slot_count(c);
     const int tg = tokens_per_frame(c) * c->block_t;
-    if (c->persistent_cache_size % tg == 0) return c->persistent_cache_size / tg * blocks_per_frame(c);
+    if (c->persistent_cache_size % tg == 0) return n_sink + c->persistent_cache_size / tg * blocks_per_frame(c);
     const int brows = c->block_t * c->block_h * c->block_w;
-    return (c->persistent_cache_size + brows - 1) / brows;
+    return n_sink + (c->persistent_cache_size + brows - 1) / brows;
 }
 
 int topk_count(const pbsa_config* c, int local_frames) {
@@ -96,6 +102,11 @@ int validate(const pbsa_config* c) {
     if (c->max_seq_len < tg) return fail(PBSA_ERR_ARG, "max_seq_len %d < one frame group (%d)", c->max_seq_len, tg);
     const float r = c->local_block_sparse_topk_ratio;
     if (!(r > 0.f && r <= 1.f)) return fail(PBSA_ERR_ARG, "local_block_sparse_topk_ratio %g not in (0, 1]", r);
+    if (c->sink_frames < 0 || c->sink_frames % c->block_t)
+        return fail(PBSA_ERR_ARG, "sink_frames %d is not a non-negative multiple of block_t %d", c->sink_frames,
+                    c->block_t);
+    if (c->sink_frames > 0 && dense_mode(c))
+        return fail(PBSA_ERR_UNSUPPORTED, "sink frames in kv_cache_mode=dense are not built");
     const int W = window_tokens(c) / tf;
     const int nlmax = W / c->block_t * blocks_per_frame(c);
     if (nlmax > 512) return fail(PBSA_ERR_UNSUPPORTED, "%d local blocks > 512", nlmax);
@@ -121,6 +132,7 @@ pbsa::Geo make_geo(const pbsa_config* c) {
     g.W = window_tokens(c) / g.tf;
     g.Wg = g.W / g.bt;
     g.S = num_slots(c);
+    g.n_sink = sink_slot_count(c);
     return g;
 }
 
@@ -128,8 +140,9 @@ int check_window(const pbsa_config* c, const pbsa::Geo& g, int q_frames, int loc
     if (q_frames < 1) return fail(PBSA_ERR_ARG, "q_frames %d < 1", q_frames);
     if ((long long)q_frames * g.tf > c->max_seq_len)
         return fail(PBSA_ERR_ARG, "q_frames*T_f = %lld > max_seq_len %d", (long long)q_frames * g.tf, c->max_seq_len);
-    if (local_frames < 1 || local_frames > g.W)
-        return fail(PBSA_ERR_ARG, "local_frames %d not in [1, %d]", local_frames, g.W);
+    // an empty window is allowed: a chunk made only of sink frames attends the slots alone
+    if (local_frames < 0 || local_frames > g.W)
+        return fail(PBSA_ERR_ARG, "local_frames %d not in [0, %d]", local_frames, g.W);
     if (ring_head < 0 || ring_head >= g.W) return fail(PBSA_ERR_ARG, "ring_head %d not in [0, %d)", ring_head, g.W);
     if (q_frames % g.bt || local_frames % g.bt || ring_head % g.bt)
         return fail(PBSA_ERR_ARG, "q_frames %d, local_frames %d and ring_head %d must be multiples of block_t %d",
@@ -261,6 +274,11 @@ int pbsa_num_slots(const pbsa_config* cfg) {
     return num_slots(cfg);
 }
 
+int pbsa_sink_slots(const pbsa_config* cfg) {
+    if (validate(cfg) != PBSA_OK) return -1;
+    return sink_slot_count(cfg);
+}
+
 int pbsa_topk_count(const pbsa_config* cfg, int local_frames) {
     if (validate(cfg) != PBSA_OK) return -1;
     if (local_frames < 0 || local_frames > window_tokens(cfg) / tokens_per_frame(cfg))
@@ -306,6 +324,46 @@ int pbsa_select_blocks(const pbsa_config* cfg, const void* q, int q_frames, cons
     if (e != cudaSuccess) return cuda_fail(e, "pool kernel launch");
     e = pbsa::launch_score_topk(g, qbar, kbar, ring_head, qb, nl, k, idx, idx_stride, cnt, scores, st);
     if (e != cudaSuccess) return cuda_fail(e, "score/top-k kernel launch");
+    return PBSA_OK;
+}
+
+int pbsa_append_frames(const pbsa_config* cfg, const void* k_new, const void* v_new, int n_frames,
+                       int first_global_frame, void* k_local, void* v_local, int ring_slot, float* kbar,
+                       void* k_pers, void* v_pers, int32_t* pers_len, float* pers_score, int32_t* pers_src,
+                       void* stream) {
+    int rc = validate(cfg);
+    if (rc != PBSA_OK) return rc;
+    const pbsa::Geo g = make_geo(cfg);
+    if (n_frames < 0 || n_frames % g.bt) return fail(PBSA_ERR_ARG, "n_frames %d is not a multiple of block_t %d", n_frames, g.bt);
+    if (first_global_frame < 0 || first_global_frame % g.bt)
+        return fail(PBSA_ERR_ARG, "first_global_frame %d is not a non-negative multiple of block_t %d",
+                    first_global_frame, g.bt);
+    if (ring_slot < 0 || ring_slot >= g.W || ring_slot % g.bt)
+        return fail(PBSA_ERR_ARG, "ring_slot %d is not a multiple of block_t in [0, %d)", ring_slot, g.W);
+    int n_sink = cfg->sink_frames - first_global_frame;
+    n_sink = n_sink < 0 ? 0 : (n_sink > n_frames ? n_frames : n_sink);
+    if (n_frames - n_sink > g.W) return fail(PBSA_ERR_ARG, "%d window frames do not fit a ring of %d", n_frames - n_sink, g.W);
+    if (n_frames == 0) return PBSA_OK;
+    REQUIRE_PTR(k_new);
+    REQUIRE_PTR(v_new);
+    if (n_frames > n_sink) {
+        REQUIRE_PTR(k_local);
+        REQUIRE_PTR(v_local);
+        OPTIONAL_PTR(kbar);
+    }
+    if (n_sink > 0) {
+        REQUIRE_PTR(k_pers);
+        REQUIRE_PTR(v_pers);
+        REQUIRE_PTR(pers_len);
+        REQUIRE_PTR(pers_score);
+        REQUIRE_PTR(pers_src);
+    }
+    cudaError_t e = pbsa::launch_append(
+        g, static_cast<const __nv_bfloat16*>(k_new), static_cast<const __nv_bfloat16*>(v_new), n_frames, n_sink,
+        first_global_frame / g.bt, static_cast<__nv_bfloat16*>(k_local), static_cast<__nv_bfloat16*>(v_local),
+        ring_slot, kbar, static_cast<__nv_bfloat16*>(k_pers), static_cast<__nv_bfloat16*>(v_pers), pers_len,
+        pers_score, pers_src, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "append kernel launch");
     return PBSA_OK;
 }
 

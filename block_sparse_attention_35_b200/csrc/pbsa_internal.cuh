@@ -24,7 +24,8 @@ struct Geo {
     int nby, nbx, nbf;  // block rows, block columns, blocks per frame group
     int W;              // frame slots of the local ring
     int Wg;             // frame groups of the ring (W / bt)
-    int S;              // persistent slots
+    int S;              // persistent slots (sink slots first)
+    int n_sink;         // sink slots at the front of the persistent store
 };
 
 // Block i of a frame group: first row and column in the frame and its valid extent.
@@ -129,6 +130,15 @@ cudaError_t launch_cache_update(const Geo& g, const __nv_bfloat16* k_local,
                                 __nv_bfloat16* k_pers, __nv_bfloat16* v_pers, int32_t* pers_len,
                                 float* pers_score, int32_t* pers_src, int32_t* upd,
                                 int32_t* n_upd, cudaStream_t st);
+
+// Appends n_frames frames (the first n_sink of them sink frames, whose first frame group is
+// global group sink_group0) to the sink slots and the ring (from ring frame ring_slot on),
+// pooling the ring frames' key means into kbar when it is not null.
+cudaError_t launch_append(const Geo& g, const __nv_bfloat16* k_new, const __nv_bfloat16* v_new,
+                          int n_frames, int n_sink, int sink_group0, __nv_bfloat16* k_local,
+                          __nv_bfloat16* v_local, int ring_slot, float* kbar, __nv_bfloat16* k_pers,
+                          __nv_bfloat16* v_pers, int32_t* pers_len, float* pers_score,
+                          int32_t* pers_src, cudaStream_t st);
 
 cudaError_t launch_wait_selftest(int32_t* status, long long timeout_ns, cudaStream_t st);
 

@@ -45,14 +45,16 @@ class pbsa_config(ctypes.Structure):
         ("persistent_cache_size", ctypes.c_int), ("max_seq_len", ctypes.c_int),
         ("kv_cache_mode", ctypes.c_int), ("use_local_block_sparse_attn", ctypes.c_int),
         ("local_block_sparse_topk_ratio", ctypes.c_float),
+        ("sink_frames", ctypes.c_int),
     ]
 
 
 def make_config(B, H, D, frame_h, frame_w, total_cache_size, local_cache_size,
                 persistent_cache_size, max_seq_len, local_block_sparse_topk_ratio,
                 use_local_block_sparse_attn=True, sparse_kv_block_size=(1, 8, 8),
-                kv_cache_mode="sparse_forcing") -> pbsa_config:
-    """Builds a pbsa_config from the SparseForcingAttention constructor arguments."""
+                kv_cache_mode="sparse_forcing", sink_frames=0) -> pbsa_config:
+    """Builds a pbsa_config from the SparseForcingAttention constructor arguments (plus
+    sink_frames, the length of the sequence's sink)."""
     modes = {"sparse_forcing": PBSA_KV_CACHE_SPARSE_FORCING, "dense": PBSA_KV_CACHE_DENSE}
     if kv_cache_mode not in modes:
         raise PBSAError(PBSA_ERR_UNSUPPORTED, f"kv_cache_mode {kv_cache_mode!r}")
@@ -60,7 +62,7 @@ def make_config(B, H, D, frame_h, frame_w, total_cache_size, local_cache_size,
     return pbsa_config(B, H, D, frame_h, frame_w, bt, bh, bw, total_cache_size,
                        local_cache_size, persistent_cache_size, max_seq_len,
                        modes[kv_cache_mode], int(bool(use_local_block_sparse_attn)),
-                       float(local_block_sparse_topk_ratio))
+                       float(local_block_sparse_topk_ratio), int(sink_frames))
 
 
 def _load():
@@ -76,6 +78,7 @@ def _load():
         "pbsa_blocks_per_frame": (I, [C]),
         "pbsa_window_frames": (I, [C]),
         "pbsa_num_slots": (I, [C]),
+        "pbsa_sink_slots": (I, [C]),
         "pbsa_topk_count": (I, [C, I]),
         "pbsa_workspace_size": (ctypes.c_size_t, [C, I, I]),
         "pbsa_last_error": (ctypes.c_char_p, []),
@@ -89,6 +92,7 @@ def _load():
                                   ctypes.c_size_t, P]),
         "pbsa_wait_selftest": (I, [P, ctypes.c_longlong, P]),
         "pbsa_pool_keys": (I, [C, P, I, I, P, P]),
+        "pbsa_append_frames": (I, [C, P, P, I, I, P, P, I, P, P, P, P, P, P, P]),
         "pbsa_select_blocks_pooled": (I, [C, P, I, P, I, I, P, I, P, P, P, ctypes.c_size_t, P]),
     }
     for name, (res, args) in sig.items():
@@ -149,6 +153,10 @@ def pbsa_window_frames(cfg) -> int:
 
 def pbsa_num_slots(cfg) -> int:
     return _lib.pbsa_num_slots(_cfg(cfg))
+
+
+def pbsa_sink_slots(cfg) -> int:
+    return _lib.pbsa_sink_slots(_cfg(cfg))
 
 
 def pbsa_topk_count(cfg, local_frames: int) -> int:
@@ -216,6 +224,17 @@ def pbsa_cache_update(cfg, k_local, v_local, local_frames, ring_head, mass_local
 
 def pbsa_wait_selftest(status, timeout_ns: int, stream=None):
     _check(_lib.pbsa_wait_selftest(_ptr(status), int(timeout_ns), _stream(stream)))
+
+
+def pbsa_append_frames(cfg, k_new, v_new, n_frames, first_global_frame, k_local, v_local,
+                       ring_slot, kbar=None, k_pers=None, v_pers=None, pers_len=None,
+                       pers_score=None, pers_src=None, stream=None):
+    """Appends frames to the cache: sink frames into their slots, the others into the ring
+    from ring_slot on, with their key means written to kbar (when given) in the same pass."""
+    _check(_lib.pbsa_append_frames(
+        _cfg(cfg), _ptr(k_new), _ptr(v_new), n_frames, first_global_frame, _ptr(k_local),
+        _ptr(v_local), ring_slot, _ptr(kbar), _ptr(k_pers), _ptr(v_pers), _ptr(pers_len),
+        _ptr(pers_score), _ptr(pers_src), _stream(stream)))
 
 
 def pbsa_pool_keys(cfg, k_local, first_slot, n_frames, kbar, stream=None):

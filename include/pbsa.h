@@ -108,6 +108,13 @@ typedef struct pbsa_config {
     int kv_cache_mode;           /* PBSA_KV_CACHE_SPARSE_FORCING or PBSA_KV_CACHE_DENSE */
     int use_local_block_sparse_attn; /* 0: every local block is attended */
     float local_block_sparse_topk_ratio; /* in (0, 1] */
+    /* Sink pattern (project page, kernel features: "local, sink, and learned top-k"; the
+     * page's constructor has no such argument, this field is this library's): the first
+     * sink_frames frames of a sequence (a multiple of block_t; 0 = no sink).  Their blocks
+     * get slots of their own at the front of the persistent store (pbsa_sink_slots), are
+     * written there by pbsa_append_frames instead of entering the window, are attended by
+     * every query and are never evicted by pbsa_cache_update. */
+    int sink_frames;
 } pbsa_config;
 
 /* ---------------------------------------------------------------- host-only queries */
@@ -119,9 +126,13 @@ PBSA_API int pbsa_blocks_per_frame(const pbsa_config* cfg);
 /* W, frame slots of the local ring (local_cache_size / T_f; total_cache_size / T_f in
  * dense mode). */
 PBSA_API int pbsa_window_frames(const pbsa_config* cfg);
-/* S, persistent slots: persistent_cache_size / (block_t * T_f) * NB when that divides,
- * else ceil(persistent_cache_size / (block_t * block_h * block_w)); 0 in dense mode. */
+/* S, persistent slots: the sink slots (pbsa_sink_slots) followed by the merged slots,
+ * persistent_cache_size / (block_t * T_f) * NB when that divides, else
+ * ceil(persistent_cache_size / (block_t * block_h * block_w)); 0 in dense mode. */
 PBSA_API int pbsa_num_slots(const pbsa_config* cfg);
+/* Sink slots at the front of the persistent store: sink_frames / block_t * NB (slot =
+ * global frame group * NB + block in group). */
+PBSA_API int pbsa_sink_slots(const pbsa_config* cfg);
 /* k, local blocks attended per query block for a window of local_frames frames:
  * N_L = local_frames / block_t * NB; k = N_L when use_local_block_sparse_attn is 0 or in dense
  * mode, else clamp(ceil(ratio * N_L), 1, N_L).  When k = N_L and no scores are asked for,
@@ -213,6 +224,30 @@ PBSA_API int pbsa_select_blocks_pooled(const pbsa_config* cfg, const void* q, in
                                        void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Frame append (the algorithm fragment: each chunk's frames enter the KV cache), fused
+ * with the key-mean cache.  The paper has no separate call for this.
+ *
+ * k_new, v_new [B, n_frames*T_f, H, D] bf16: frames first_global_frame,
+ * first_global_frame + 1, ... of the sequence (n_frames and first_global_frame multiples
+ * of block_t).  Frames below cfg->sink_frames are sink frames: each of their blocks is
+ * written whole into sink slot (global frame group * NB + block in group) of
+ * key_persistent / value_persistent (rows past its length zeroed) with pers_len = token
+ * count, pers_score = 0, pers_src = slot; sink frames come before every window frame of a
+ * sequence.  Every other frame f goes to ring frame (ring_slot + f - n_sink) % W of
+ * k_local / v_local, n_sink being the number of sink frames in this call
+ * (clamp(sink_frames - first_global_frame, 0, n_frames)); when kbar is not NULL the mean
+ * key of each of their blocks is written to kbar as pbsa_pool_keys does, in the same
+ * pass.  One read of the new frames, one write of each copy.  Persistent pointers may be
+ * NULL when no sink frame is appended.  ring_slot is a multiple of block_t in [0, W) and
+ * the window frames appended fit in the ring (n_frames - n_sink <= W).
+ */
+PBSA_API int pbsa_append_frames(const pbsa_config* cfg, const void* k_new, const void* v_new,
+                                int n_frames, int first_global_frame, void* k_local, void* v_local,
+                                int ring_slot, float* kbar, void* k_pers, void* v_pers,
+                                int32_t* pers_len, float* pers_score, int32_t* pers_src,
+                                void* stream);
+
+/*
  * PBSA forward.  (pith.science abstract; project page call attn(query, key_persistent,
  * value_persistent, key_local, value_local).)
  *
@@ -264,10 +299,10 @@ PBSA_API int pbsa_attn_bwd(const pbsa_config* cfg, const void* q, int q_frames,
  * Window slide and persistent merge (pith.science abstract: persistent blocks are
  * compressed, preserved and updated; algorithm fragment: the t=0 pass updates P and L).
  *
- * The oldest n_evict_frames frames of the window leave it.  Candidates are the occupied
- * slots (score pers_score) followed by the evicted blocks in logical id order (score
+ * The oldest n_evict_frames frames of the window leave it.  The sink slots take no part.
+ * Candidates are the occupied merged slots (score pers_score) followed by the evicted blocks in logical id order (score
  * mass_local of their physical block).  Ordered by score descending, ties by that
- * candidate order, the first min(S, #candidates) are kept.  Kept slots stay in place;
+ * candidate order, the first min(S - sink slots, #candidates) are kept.  Kept slots stay in place;
  * the free slots (empty ones ascending, then dropped ones ascending) receive the kept
  * evicted blocks in id order: tokens copied frame by frame in raster order, pers_len =
  * token count, pers_score = the block's mass, pers_src = global frame group * NB + block

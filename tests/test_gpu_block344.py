@@ -127,3 +127,18 @@ def test_344_wrapper_rollout_against_decode_step(cuda_dev):
               for _ in range(wl.chunks)]
     a, _, admitted = _run_rollout(wl, cuda_dev, wl.chunks, lambda s: chunks[s])
     assert sum(admitted) >= a.S
+
+
+def test_344_rollout_with_a_sink_group(cuda_dev):
+    """[3,4,4] blocks with the first 3-frame group as the sink: chunk 0 is all sink, so its
+    queries attend the sink slots alone (an empty window); later chunks add the window and
+    the merge, which never touches the 20 sink slots.  Replayed step by step by the oracle."""
+    wl = dataclasses.replace(B344, B=1, H=1, chunks=5)
+    gen = torch.Generator().manual_seed(7)
+    shape = (1, wl.q_frames * wl.tokens_per_frame, 1, wl.D)
+    chunks = [tuple(torch.randn(shape, generator=gen).to(torch.bfloat16) for _ in range(3))
+              for _ in range(wl.chunks)]
+    a, _, admitted = _run_rollout(wl, cuda_dev, wl.chunks, lambda s: chunks[s], sink_frames=3)
+    assert a.n_sink == 20 and a.S == 40
+    assert (a.pers_src[0, 0, :20].cpu() == torch.arange(20)).all()
+    assert sum(admitted) > 0

@@ -40,14 +40,15 @@ def _state_from_gpu(a, W, tf, nbf):
         a.pers_score.cpu().double().numpy(), a.pers_src.cpu().numpy(), a.first_frame_global)
 
 
-def _run_rollout(wl, dev, chunks, chunk_fn):
+def _run_rollout(wl, dev, chunks, chunk_fn, sink_frames=0):
     a = SparseForcingAttention(wl.B, wl.H, wl.D, wl.frame_h, wl.frame_w, wl.total_cache_size,
                                wl.local_cache_size, wl.persistent_cache_size,
                                sparse_kv_block_size=wl.block, max_seq_len=wl.max_seq_len,
                                local_block_sparse_topk_ratio=wl.topk_ratio,
-                               chunk_frames=wl.q_frames, device=dev)
+                               chunk_frames=wl.q_frames, sink_frames=sink_frames, device=dev)
     W, tf, nbf, S = a.W, a.tf, a.nbf, a.S
     bt, bh, bw = wl.block
+    n_sink = a.n_sink
     exact_frac, admitted = [], []
     for step in range(chunks):
         q, k, v = chunk_fn(step)
@@ -61,12 +62,18 @@ def _run_rollout(wl, dev, chunks, chunk_fn):
         # ---- the oracle's step on the same state, with the GPU's selection (near-ties may
         # legitimately differ; the selection itself is checked against the oracle's scores)
         st1, o = orc.decode_step(st0, f64(q), f64(k), f64(v), wl.topk_ratio, W, wl.frame_h,
-                                 wl.frame_w, idx=idx[..., :P_k(a, lf)], bh=bh, bw=bw, bt=bt)
-        kwin = np.concatenate([st0.win_k, f64(k)], 1)
-        vwin = np.concatenate([st0.win_v, f64(v)], 1)
-        _, sc_o = orc.select_blocks(f64(q), kwin, wl.frame_h, wl.frame_w, wl.topk_ratio, bh=bh, bw=bw, bt=bt)
+                                 wl.frame_w, idx=idx[..., :P_k(a, lf)], bh=bh, bw=bw, bt=bt,
+                                 sink_frames=sink_frames)
+        appended = orc.append_frames(st0, f64(k), f64(v), sink_frames, wl.frame_h, wl.frame_w,
+                                     bh, bw, bt)
+        kwin, vwin = appended.win_k, appended.win_v
+        assert np.array_equal(a.pers_len.cpu().numpy(), appended.pers_len)
+        assert np.array_equal(f64(a.k_pers), appended.k_pers)
         kk = P_k(a, lf)
-        exact_frac.append(check_topk(idx[..., :kk], a.cnt.cpu().numpy(), sc_o, kk))
+        if kk:
+            _, sc_o = orc.select_blocks(f64(q), kwin, wl.frame_h, wl.frame_w, wl.topk_ratio,
+                                        bh=bh, bw=bw, bt=bt)
+            exact_frac.append(check_topk(idx[..., :kk], a.cnt.cpu().numpy(), sc_o, kk))
         assert_close_bf16(f64(a.out), o["O"], f"step {step} out")
         assert np.abs(a.lse.cpu().numpy() - o["lse"]).max() <= LSE_ABS
         ps1 = a.pers_score.cpu().double().numpy()
@@ -81,9 +88,10 @@ def _run_rollout(wl, dev, chunks, chunk_fn):
         if n_ev:
             ups = [tuple(x) for x in a.upd[0, 0, :nup[0]].cpu().numpy()]
             # decisions on the GPU's own masses must match the oracle's merge exactly
-            r = orc.cache_update(st0.k_pers, st0.v_pers, st0.pers_len, ps1, st0.pers_src, kwin,
-                                 vwin, ml1, n_ev, st0.first_frame_global, wl.frame_h, wl.frame_w,
-                                 bh, bw, bt)
+            r = orc.cache_update(appended.k_pers, appended.v_pers, appended.pers_len, ps1,
+                                 appended.pers_src, kwin, vwin, ml1, n_ev,
+                                 appended.first_frame_global, wl.frame_h, wl.frame_w, bh, bw, bt,
+                                 n_sink)
             assert ups == r["updates"][0][0], f"step {step}"
             assert np.array_equal(a.pers_len.cpu().numpy(), r["pers_len"])
             assert np.array_equal(a.pers_src.cpu().numpy(), r["pers_src"])
@@ -91,10 +99,12 @@ def _run_rollout(wl, dev, chunks, chunk_fn):
             assert np.array_equal(f64(a.v_pers), r["v_pers"])
             # and the oracle's own step (its masses) decides the same wherever the keep/drop
             # margin exceeds 1e-3
-            cand = [o["pers_score_before_merge"][0, 0, s] for s in range(S) if st0.pers_len[0, 0, s] > 0]
+            cand = [o["pers_score_before_merge"][0, 0, s] for s in range(n_sink, S)
+                    if appended.pers_len[0, 0, s] > 0]
             cand += list(o["win_mass_before_merge"][0, 0, :n_ev // bt * nbf])
             srt = sorted(cand, reverse=True)
-            margin = (srt[S - 1] - srt[S]) if len(srt) > S else np.inf
+            Sm = S - n_sink
+            margin = (srt[Sm - 1] - srt[Sm]) if len(srt) > Sm else np.inf
             if margin > 1e-3:
                 assert o["updates"][0][0] == ups, f"step {step}: decision differs at margin {margin}"
                 assert np.array_equal(st1.pers_len, a.pers_len.cpu().numpy())
@@ -131,3 +141,15 @@ def test_rollout_hot_blocks_turn_the_cache_over(cuda_dev):
     full_at = next(i for i in range(len(admitted)) if sum(admitted[:i + 1]) >= a.S)
     assert sum(admitted[full_at + 1:]) > 0, f"no admissions after the cache filled: {admitted}"
     print(f"hot rollout: admissions {admitted}")
+
+
+def test_rollout_with_a_sink_frame(cuda_dev):
+    """Decode geometry (one head), the first frame of the sequence as the sink: its 28
+    blocks live in sink slots from chunk 0 on, are attended by every query, and no merge
+    touches them; 6 chunks, every step replayed by the oracle."""
+    wl = dataclasses.replace(WORKLOADS["rollout"], H=1, chunks=6)
+    a, _, admitted = _run_rollout(wl, cuda_dev, wl.chunks, lambda s: rollout_chunk_hot(wl, s),
+                                  sink_frames=1)
+    assert a.n_sink == 28
+    assert (a.pers_len[0, 0, :28] > 0).all() and (a.pers_src[0, 0, :28].cpu() == torch.arange(28)).all()
+    assert sum(admitted) > 0
