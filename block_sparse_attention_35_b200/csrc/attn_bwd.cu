@@ -317,6 +317,18 @@ __device__ __forceinline__ void dkdv_body(const BwdKernelArgs& ka, const int cta
             }
         }
         __syncwarp();
+        // in-block coordinates of this lane's four rows of a query tile (rows lane + 32 u:
+        // u = 0, 1 in its first query block, u = 2, 3 in its second); fixed for the CTA
+        int rt[4], ry[4], rx[4];
+        bool rin[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int rr = (lane + 32 * u) & 63;
+            rx[u] = rr % g.bw;
+            ry[u] = (rr / g.bw) % g.bh;
+            rt[u] = rr / (g.bw * g.bh);
+            rin[u] = rr < g.brows;
+        }
         int issued = 0;
         for (int j = 0; j < n_items; ++j) {
             const int st = j % kNst;
@@ -326,17 +338,21 @@ __device__ __forceinline__ void dkdv_body(const BwdKernelArgs& ka, const int cta
             // masks padding rows
             float l2v[4], dlv[4];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int r = lane + 32 * u;
-                const int hq = r >> 6, qb = 2 * qt + hq;
-                l2v[u] = CUDART_INF_F;
-                dlv[u] = 0.f;
+            for (int hq = 0; hq < 2; ++hq) {
+                const int qb = 2 * qt + hq;
+                BlockBox qbb = {0, 0, 0, 0};
+                size_t base = 0;
                 if (qb < qb_total) {
-                    const BlockBox qbb = block_box(g, qb % g.nbf);
-                    int tt, y, x;
-                    if (block_row(g, qbb, r & 63, &tt, &y, &x)) {
-                        const size_t t = (size_t)bh * nq + (size_t)((qb / g.nbf) * g.bt + tt) * g.tf +
-                                         (qbb.y0 + y) * g.fw + qbb.x0 + x;
+                    qbb = block_box(g, qb % g.nbf);
+                    base = (size_t)bh * nq + (size_t)(qb / g.nbf) * g.bt * g.tf + qbb.y0 * g.fw + qbb.x0;
+                }
+#pragma unroll
+                for (int v = 0; v < 2; ++v) {
+                    const int u = 2 * hq + v;
+                    l2v[u] = CUDART_INF_F;
+                    dlv[u] = 0.f;
+                    if (qb < qb_total && rin[u] && ry[u] < qbb.hv && rx[u] < qbb.wv) {
+                        const size_t t = base + (size_t)rt[u] * g.tf + ry[u] * g.fw + rx[u];
                         l2v[u] = a.lse[t] * kLog2e;
                         dlv[u] = a.delta[t];
                     }
@@ -475,8 +491,10 @@ __device__ __forceinline__ void dkdv_body(const BwdKernelArgs& ka, const int cta
                     float p[4], d[4];
 #pragma unroll
                     for (int u = 0; u < 4; ++u) {
+                        // p is exactly 0 off the selection; dP^T there is finite (key rows past
+                        // a slot's length are finite), so dS^T is exactly 0 as well
                         p[u] = sel ? fast_exp2(__uint_as_float(sv[4 * e4 + u]) * sl2 - ls[u]) : 0.f;
-                        d[u] = sel ? p[u] * (__uint_as_float(pv[4 * e4 + u]) - ds[u]) : 0.f;
+                        d[u] = p[u] * (__uint_as_float(pv[4 * e4 + u]) - ds[u]);
                     }
                     pk[8 * sc + 2 * e4] = pack_bf16x2(p[0], p[1]);
                     pk[8 * sc + 2 * e4 + 1] = pack_bf16x2(p[2], p[3]);
@@ -554,7 +572,7 @@ __device__ __forceinline__ void dkdv_body(const BwdKernelArgs& ka, const int cta
 
 // ========================================================================== dQ
 struct DqPlan {
-    uint32_t q, dq_o, k, v, grp_row, uni_blk, uni_bits, blk_mask, bars, misc, total;
+    uint32_t q, dq_o, k, v, grp_row, tile_mask, uni_blk, uni_bits, blk_mask, bars, misc, total;
 };
 
 __host__ __device__ inline DqPlan dq_plan(int D, int S, int ucap, int nbf) {
@@ -565,7 +583,8 @@ __host__ __device__ inline DqPlan dq_plan(int D, int S, int ucap, int nbf) {
     p.k = p.dq_o + nh * kHalf;
     p.v = p.k + kNst * nh * kHalf;
     p.grp_row = p.v + kNst * nh * kHalf;
-    p.uni_blk = p.grp_row + 4u * 8u * S;
+    p.tile_mask = p.grp_row + 4u * 8u * S;              // [16-group tiles][4] valid key columns
+    p.uni_blk = p.tile_mask + 16u * ((8u * S + 15u) / 16u);
     p.uni_bits = p.uni_blk + 4u * ucap;
     p.blk_mask = (p.uni_bits + 4u * ucap + 7u) & ~7u;  // [nbf] valid rows of each block
     p.bars = p.blk_mask + 8u * nbf;
@@ -594,6 +613,7 @@ __device__ __forceinline__ void dq_body(const BwdKernelArgs& ka, const int tile,
     uint8_t* sK = sm + PL.k;
     uint8_t* sV = sm + PL.v;
     int32_t* grp_row = reinterpret_cast<int32_t*>(sm + PL.grp_row);
+    uint32_t* tile_mask = reinterpret_cast<uint32_t*>(sm + PL.tile_mask);
     int32_t* uni_blk = reinterpret_cast<int32_t*>(sm + PL.uni_blk);
     int32_t* uni_bits = reinterpret_cast<int32_t*>(sm + PL.uni_bits);
     uint64_t* blk_mask = reinterpret_cast<uint64_t*>(sm + PL.blk_mask);
@@ -638,6 +658,19 @@ __device__ __forceinline__ void dq_body(const BwdKernelArgs& ka, const int tile,
     if (warp == 0) {
         const int G = build_groups(a.pers_len, bh, S, grp_row, a.status);
         if (lane == 0) misc[2] = G;
+        __syncwarp();
+        // valid key columns of each 16-group tile, one 32-bit word per 4 groups
+        for (int w = lane; w < 4 * ((G + 15) / 16); w += 32) {
+            uint32_t m = 0;
+            for (int gq = 0; gq < 4; ++gq) {
+                const int gi = 4 * w + gq;
+                if (gi < G) {
+                    const int nv = group_rows(grp_row[gi]);
+                    m |= (nv >= 8 ? 0xffu : ((1u << nv) - 1u)) << (8 * gq);
+                }
+            }
+            tile_mask[w] = m;
+        }
     }
     if (warp == 1 && lane == 0) {
         const int c0 = min(max(a.cnt[(size_t)bh * qb_total + qb0], 0), a.idx_stride);
@@ -798,16 +831,7 @@ __device__ __forceinline__ void dq_body(const BwdKernelArgs& ka, const int tile,
             // valid-column mask of this warp's 32 key columns
             uint32_t vmask;
             if (it < n_pt) {
-                // the warp's 32 columns are groups 16 it + c0 / 8 .. + 3 of the stream
-                vmask = 0u;
-#pragma unroll
-                for (int gq = 0; gq < kCw / 8; ++gq) {
-                    const int gi = 16 * it + c0 / 8 + gq;
-                    if (gi < G) {
-                        const int nv = group_rows(grp_row[gi]);
-                        vmask |= (nv >= 8 ? 0xffu : ((1u << nv) - 1u)) << (8 * gq);
-                    }
-                }
+                vmask = tile_mask[4 * it + cg];   // the warp's 32 columns: groups 16 it + 4 cg ..
             } else {
                 const int u = 2 * (it - n_pt) + kh;
                 const bool has = u < U;
@@ -829,8 +853,8 @@ __device__ __forceinline__ void dq_body(const BwdKernelArgs& ka, const int tile,
 #pragma unroll
                     for (int u = 0; u < 2; ++u) {
                         const bool valid = (vmask >> (16 * sc + e + u)) & 1u;
-                        const float p = fast_exp2(__uint_as_float(sv[e + u]) * sl2 - lse2);
-                        dsv[u] = valid ? p * (__uint_as_float(pv[e + u]) - dl) : 0.f;
+                        const float p = valid ? fast_exp2(__uint_as_float(sv[e + u]) * sl2 - lse2) : 0.f;
+                        dsv[u] = p * (__uint_as_float(pv[e + u]) - dl);
                     }
                     dk[8 * sc + e / 2] = pack_bf16x2(dsv[0], dsv[1]);
                 }

@@ -488,13 +488,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         const int wq = warp & 3;          // lane quarter
         const int nX = X ? n_side1 : n_side0;
         const int hq = r >> 6;
-        const int qbr = qblock(X, hq);
-        const int qbv = qbr >= 0 ? qbr : 0;
-        const BlockBox qbb = block_box(g, qbv % g.nbf);
-        int qt, qy, qx;
-        const bool row_valid = block_row(g, qbb, r & 63, &qt, &qy, &qx) && qbr >= 0;
-        // token of this row in the chunk
-        const size_t q_tok = (size_t)((qbv / g.nbf) * g.bt + qt) * g.tf + (qbb.y0 + qy) * g.fw + qbb.x0 + qx;
+        // token of this row in the chunk, or -1 for a padding row (computed in the epilogue,
+        // where it is needed, so that nothing of it stays live in the loop)
+        auto row_token = [&]() -> long long {
+            const int qbr = qblock(X, hq);
+            if (qbr < 0) return -1;
+            const BlockBox qbb = block_box(g, qbr % g.nbf);
+            int qt, qy, qx;
+            if (!block_row(g, qbb, r & 63, &qt, &qy, &qx)) return -1;
+            return (long long)((qbr / g.nbf) * g.bt + qt) * g.tf + (qbb.y0 + qy) * g.fw + qbb.x0 + qx;
+        };
         const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
         const uint32_t s_col = 128 * X, o_col = 256 + 128 * X;
         const float sl2 = kLog2e / sqrtf(static_cast<float>(D));
@@ -671,6 +674,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                 }
             }
             const float lse2 = (l > 0.f) ? m + fast_log2(l) : -CUDART_INF_F;
+            const long long q_tok = row_token();
+            const bool row_valid = q_tok >= 0;
             if (row_valid) a.lse[(size_t)bh * a.q_frames * g.tf + q_tok] = lse2 * 0.6931471805599453f;
             fence_proxy_async_smem();
             named_bar_sync(bar_id, 128);

@@ -52,14 +52,15 @@ __host__ __device__ inline bool block_row(const Geo& g, const BlockBox& bb, int 
     return r < g.brows && *y < bb.hv && *x < bb.wv;
 }
 
-// Valid rows of block i as a 64-bit mask over its box rows.
+// Valid rows of block i as a 64-bit mask over its box rows (the rows block_row accepts),
+// built with shifts: wv bits per row of the frame, hv rows per frame, bt frames.
 __host__ __device__ inline uint64_t block_rows_mask(const Geo& g, int i) {
     const BlockBox bb = block_box(g, i);
+    const uint64_t row = bb.wv >= 64 ? ~0ull : ((1ull << bb.wv) - 1ull);
+    uint64_t plane = 0;
+    for (int y = 0; y < bb.hv; ++y) plane |= row << (y * g.bw);
     uint64_t m = 0;
-    for (int r = 0; r < g.brows; ++r) {
-        int t, y, x;
-        if (block_row(g, bb, r, &t, &y, &x)) m |= 1ull << r;
-    }
+    for (int t = 0; t < g.bt; ++t) m |= plane << (t * g.bh * g.bw);
     return m;
 }
 
