@@ -19,7 +19,9 @@
 //  3. bwd_kernel, dQ CTAs (dq_body): one CTA per query tile (the forward's tiling); per key
 //     tile S = Q K^T and dP = dO V^T in TMEM, the element warps (a query-row quarter and 32
 //     key columns each) form dS, write it as bf16 over S, and a TS MMA accumulates
-//     dQ += dS K (K read MN-major).
+//     dQ += dS K (K read MN-major).  S is double-buffered in TMEM (S, S', dP, dQ = 512
+//     columns) and the element warps release dP as soon as they have read it, so the next
+//     key tile's S and dP are computed while the current tile's dS is formed.
 // Warp roles in both parts: warps 0-15 elementwise (P, dS), warp 16 TMA producer, warp 17
 // MMA.  The MMA thread issues the next tile's S / dP right after the current tile's
 // gradient MMAs (the tensor pipe runs them in issue order), so only the element warps'
@@ -575,14 +577,18 @@ struct DqPlan {
     uint32_t q, dq_o, k, v, grp_row, tile_mask, uni_blk, uni_bits, blk_mask, bars, misc, total;
 };
 
+// dQ CTAs: K tiles live from S = Q K^T until the dQ MMA of their tile (three stages), V
+// tiles only until dP = dO V^T (one stage).
+constexpr int kDqKst = 3, kDqVst = 1;
+
 __host__ __device__ inline DqPlan dq_plan(int D, int S, int ucap, int nbf) {
     DqPlan p;
     const uint32_t nh = D / 64;
     p.q = 0;
     p.dq_o = p.q + nh * kHalf;
     p.k = p.dq_o + nh * kHalf;
-    p.v = p.k + kNst * nh * kHalf;
-    p.grp_row = p.v + kNst * nh * kHalf;
+    p.v = p.k + kDqKst * nh * kHalf;
+    p.grp_row = p.v + kDqVst * nh * kHalf;
     p.tile_mask = p.grp_row + 4u * 8u * S;              // [16-group tiles][4] valid key columns
     p.uni_blk = p.tile_mask + 16u * ((8u * S + 15u) / 16u);
     p.uni_bits = p.uni_blk + 4u * ucap;
@@ -599,7 +605,8 @@ template <int D>
 __device__ __forceinline__ void dq_body(const BwdKernelArgs& ka, const int tile, const int h, const int b) {
     constexpr int NH = D / 64;
     constexpr uint32_t TILE = NH * kHalf;
-    constexpr uint32_t kTmS = 0, kTmP = 128, kTmQ = 256;
+    // TMEM: two S buffers (tile t in buffer t & 1), dP, dQ
+    constexpr uint32_t kTmS = 0, kTmP = 256, kTmQ = 384;
     const BwdArgs& a = ka.a;
     const Geo& g = a.g;
     extern __shared__ uint8_t smem_raw[];
@@ -621,13 +628,15 @@ __device__ __forceinline__ void dq_body(const BwdKernelArgs& ka, const int tile,
     int* misc = reinterpret_cast<int*>(sm + PL.misc);
     volatile int* abort_flag = misc + 1;
     uint64_t* q_full = &bars[0];
-    uint64_t* k_full = &bars[1];    // [kNst]
-    uint64_t* v_full = &bars[3];    // [kNst]
-    uint64_t* kv_empty = &bars[5];  // [kNst]
-    uint64_t* sdp_full = &bars[7];
-    uint64_t* ds_full = &bars[8];
-    uint64_t* dq_done = &bars[9];
-    uint64_t* drain = &bars[10];
+    uint64_t* k_full = &bars[1];    // [kDqKst]
+    uint64_t* k_empty = &bars[4];   // [kDqKst]
+    uint64_t* v_full = &bars[7];
+    uint64_t* v_empty = &bars[8];
+    uint64_t* sdp_full = &bars[9];  // S and dP of a tile computed
+    uint64_t* dp_free = &bars[10];  // every element warp has read dP (kElemWarps arrivals)
+    uint64_t* ds_full = &bars[11];  // dS written (kElemWarps arrivals)
+    uint64_t* dq_done = &bars[12];
+    uint64_t* drain = &bars[13];
 
     const int bh = b * g.H + h;
     const int qb_total = a.q_frames / g.bt * g.nbf;
@@ -640,12 +649,14 @@ __device__ __forceinline__ void dq_body(const BwdKernelArgs& ka, const int tile,
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
-        for (int s = 0; s < kNst; ++s) {
+        for (int s = 0; s < kDqKst; ++s) {
             mbar_init(&k_full[s], 1);
-            mbar_init(&v_full[s], 1);
-            mbar_init(&kv_empty[s], 1);
+            mbar_init(&k_empty[s], 1);
         }
+        mbar_init(v_full, 1);
+        mbar_init(v_empty, 1);
         mbar_init(sdp_full, 1);
+        mbar_init(dp_free, kElemWarps);
         mbar_init(ds_full, kElemWarps);
         mbar_init(dq_done, 1);
         mbar_init(drain, 1);
@@ -723,45 +734,51 @@ __device__ __forceinline__ void dq_body(const BwdKernelArgs& ka, const int tile,
                     tma_load_5d(sDO + hh * kHalf + hb * (kHalf / 2), &a.tm_do, q_full, hh * 64, h, qbb.x0, qbb.y0, f0);
                 }
             }
+            // K of tile it into stage it % 3 once the dQ MMA of tile it - 3 is done; V of tile
+            // it into the single V stage once dP of tile it - 1 is done
             int issued = 0;
             for (int it = 0; it < n_tiles; ++it) {
-                const int st = it % kNst;
-                if (it >= kNst && !mbar_wait(&kv_empty[st], ((it / kNst) - 1) & 1, abort_flag, a.status)) break;
+                const int st = it % kDqKst;
+                if (it >= kDqKst && !mbar_wait(&k_empty[st], ((it / kDqKst) - 1) & 1, abort_flag, a.status)) break;
                 uint8_t* dk = sK + st * TILE;
-                uint8_t* dv = sV + st * TILE;
                 const uint32_t tile_bytes = it < n_pt ? TILE : 2 * NH * box_bytes;
                 mbar_arrive_expect_tx(&k_full[st], tile_bytes);
-                mbar_arrive_expect_tx(&v_full[st], tile_bytes);
                 if (it < n_pt) {
-                    for (int c = 0; c < 16; ++c) {
-                        const int row = grp_row[min(it * 16 + c, G - 1)] & ~7;
-                        for (int hh = 0; hh < NH; ++hh) {
-                            tma_load_2d(dk + hh * kHalf + c * 1024, &a.tm_kp, &k_full[st], hh * 64, row);
-                            tma_load_2d(dv + hh * kHalf + c * 1024, &a.tm_vp, &v_full[st], hh * 64, row);
-                        }
-                    }
+                    tma_load_groups16<NH>(dk, kHalf, &a.tm_kp, &a.tm_kp64, grp_row, it * 16, G, &k_full[st]);
                 } else {
                     const int j = it - n_pt;
                     for (int hb = 0; hb < 2; ++hb) {
                         const int L = uni_blk[min(2 * j + hb, U - 1)];
                         const BlockBox kbb = block_box(g, L % g.nbf);
                         const int fr = b * g.W + (a.ring_head + (L / g.nbf) * g.bt) % g.W;
-                        for (int hh = 0; hh < NH; ++hh) {
+                        for (int hh = 0; hh < NH; ++hh)
                             tma_load_5d(dk + hh * kHalf + hb * (kHalf / 2), &a.tm_kl, &k_full[st], hh * 64, h,
                                         kbb.x0, kbb.y0, fr);
-                            tma_load_5d(dv + hh * kHalf + hb * (kHalf / 2), &a.tm_vl, &v_full[st], hh * 64, h,
+                    }
+                }
+                if (it >= 1 && !mbar_wait(v_empty, (it - 1) & 1, abort_flag, a.status)) { ++issued; break; }
+                mbar_arrive_expect_tx(v_full, tile_bytes);
+                if (it < n_pt) {
+                    tma_load_groups16<NH>(sV, kHalf, &a.tm_vp, &a.tm_vp64, grp_row, it * 16, G, v_full);
+                } else {
+                    const int j = it - n_pt;
+                    for (int hb = 0; hb < 2; ++hb) {
+                        const int L = uni_blk[min(2 * j + hb, U - 1)];
+                        const BlockBox kbb = block_box(g, L % g.nbf);
+                        const int fr = b * g.W + (a.ring_head + (L / g.nbf) * g.bt) % g.W;
+                        for (int hh = 0; hh < NH; ++hh)
+                            tma_load_5d(sV + hh * kHalf + hb * (kHalf / 2), &a.tm_vl, v_full, hh * 64, h,
                                         kbb.x0, kbb.y0, fr);
-                        }
                     }
                 }
                 ++issued;
             }
             if (*abort_flag) {
+                // let the copies already issued land before the CTA leaves
                 mbar_wait_drain(q_full, 0, 100000000ull);
-                for (int it = max(0, issued - kNst); it < issued; ++it) {
-                    mbar_wait_drain(&k_full[it % kNst], (it / kNst) & 1, 100000000ull);
-                    mbar_wait_drain(&v_full[it % kNst], (it / kNst) & 1, 100000000ull);
-                }
+                for (int it = max(0, issued - kDqKst); it < issued; ++it)
+                    mbar_wait_drain(&k_full[it % kDqKst], (it / kDqKst) & 1, 100000000ull);
+                if (issued > 0) mbar_wait_drain(v_full, (issued - 1) & 1, 100000000ull);
             }
         }
     } else if (warp == kMmaWarp) {
@@ -769,34 +786,56 @@ __device__ __forceinline__ void dq_body(const BwdKernelArgs& ka, const int tile,
             constexpr uint32_t id_s = idesc_bf16(128, 128, false, false);
             constexpr uint32_t id_g = idesc_bf16(128, D, false, true);
             bool ok = mbar_wait(q_full, 0, abort_flag, a.status);
-            const uint32_t qbase = smem_u32(sQ), obase = smem_u32(sDO);
-            for (int it = 0; ok && it < n_tiles; ++it) {
-                const int st = it % kNst;
-                if (!mbar_wait(&k_full[st], (it / kNst) & 1, abort_flag, a.status)) { ok = false; break; }
-                if (!mbar_wait(&v_full[st], (it / kNst) & 1, abort_flag, a.status)) { ok = false; break; }
-                // the previous tile's dQ MMAs read dS from TMEM before the next S lands there:
-                // MMAs issued by this thread run in issue order
+            const uint32_t qbase = smem_u32(sQ), obase = smem_u32(sDO), vb = smem_u32(sV);
+            // S(t) = Q K(t)^T into S buffer t & 1; dP(t) = dO V(t)^T; both then committed to
+            // sdp_full.  Per tile t the issue order is S(t+1), dP(t+1), dQ += dS(t) K(t): the
+            // next tile's S and dP run while the element warps work on tile t (dP(t+1) only once
+            // every element warp has read dP(t)); the tensor pipe executes one thread's MMAs in
+            // issue order, so S(t+2) never overwrites dS(t) before dQ(t) has read it.
+            auto issue_s = [&](int t) -> bool {
+                const int st = t % kDqKst;
+                if (!mbar_wait(&k_full[st], (t / kDqKst) & 1, abort_flag, a.status)) return false;
                 tc_fence_after();
-                const uint32_t kb = smem_u32(sK + st * TILE), vb = smem_u32(sV + st * TILE);
+                const uint32_t kb = smem_u32(sK + st * TILE);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
-                    umma_ss(tmem + kTmS, sdesc_make(sdesc_lo(qbase, 16) + (off >> 4)), sdesc_make(sdesc_lo(kb, 16) + (off >> 4)), id_s, kk > 0);
+                    umma_ss(tmem + kTmS + 128 * (t & 1), sdesc_make(sdesc_lo(qbase, 16) + (off >> 4)),
+                            sdesc_make(sdesc_lo(kb, 16) + (off >> 4)), id_s, kk > 0);
                 }
+                return true;
+            };
+            auto issue_dp = [&](int t) -> bool {
+                if (!mbar_wait(v_full, t & 1, abort_flag, a.status)) return false;
+                tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
-                    umma_ss(tmem + kTmP, sdesc_make(sdesc_lo(obase, 16) + (off >> 4)), sdesc_make(sdesc_lo(vb, 16) + (off >> 4)), id_s, kk > 0);
+                    umma_ss(tmem + kTmP, sdesc_make(sdesc_lo(obase, 16) + (off >> 4)),
+                            sdesc_make(sdesc_lo(vb, 16) + (off >> 4)), id_s, kk > 0);
                 }
+                umma_commit(v_empty);
                 umma_commit(sdp_full);
+                return true;
+            };
+            if (ok && n_tiles > 0) ok = issue_s(0) && issue_dp(0);
+            for (int it = 0; ok && it < n_tiles; ++it) {
+                if (it + 1 < n_tiles) {
+                    if (!issue_s(it + 1)) { ok = false; break; }
+                    if (!mbar_wait(dp_free, it & 1, abort_flag, a.status)) { ok = false; break; }
+                    if (!issue_dp(it + 1)) { ok = false; break; }
+                }
                 if (!mbar_wait(ds_full, it & 1, abort_flag, a.status)) { ok = false; break; }
                 tc_fence_after();
+                const int st = it % kDqKst;
+                const uint32_t kb = smem_u32(sK + st * TILE);
+                const uint32_t s_buf = tmem + kTmS + 128 * (it & 1);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    umma_ts(tmem + kTmQ, tmem + kTmS + packed_col(kk), sdesc_make(sdesc_lo(kb, kHalf) + kk * 128), id_g,
+                    umma_ts(tmem + kTmQ, s_buf + packed_col(kk), sdesc_make(sdesc_lo(kb, kHalf) + kk * 128), id_g,
                             (it > 0 || kk > 0) ? 1u : 0u);
                 umma_commit(dq_done);
-                umma_commit(&kv_empty[st]);
+                umma_commit(&k_empty[st]);
             }
             if (!ok) {
                 umma_commit(drain);
@@ -840,12 +879,26 @@ __device__ __forceinline__ void dq_body(const BwdKernelArgs& ka, const int tile,
                 // columns c0.. are the block's box rows (c0 & 63) + e
                 vmask = sel ? static_cast<uint32_t>(blk_mask[L % g.nbf] >> (c0 & 63)) : 0u;
             }
+            // dP first: once every element warp holds its dP columns the MMA thread may
+            // compute the next tile's dP into the same columns
+            const uint32_t s_buf = kTmS + 128 * (it & 1);
+            float dpm[kCw];
+            {
+                uint32_t pv[kCw];
+                tmem_ld16(tmem + lane_base + kTmP + c0, *reinterpret_cast<uint32_t(*)[16]>(pv));
+                tmem_ld16(tmem + lane_base + kTmP + c0 + 16, *reinterpret_cast<uint32_t(*)[16]>(pv + 16));
+                tmem_ld_wait();
+#pragma unroll
+                for (int e = 0; e < kCw; ++e) dpm[e] = __uint_as_float(pv[e]) - dl;
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(dp_free);
             uint32_t dk[kCw / 2];
 #pragma unroll
             for (int sc = 0; sc < kCw / 16; ++sc) {
-                uint32_t sv[16], pv[16];
-                tmem_ld16(tmem + lane_base + kTmS + c0 + 16 * sc, sv);
-                tmem_ld16(tmem + lane_base + kTmP + c0 + 16 * sc, pv);
+                uint32_t sv[16];
+                tmem_ld16(tmem + lane_base + s_buf + c0 + 16 * sc, sv);
                 tmem_ld_wait();
 #pragma unroll
                 for (int e = 0; e < 16; e += 2) {
@@ -854,12 +907,12 @@ __device__ __forceinline__ void dq_body(const BwdKernelArgs& ka, const int tile,
                     for (int u = 0; u < 2; ++u) {
                         const bool valid = (vmask >> (16 * sc + e + u)) & 1u;
                         const float p = valid ? fast_exp2(__uint_as_float(sv[e + u]) * sl2 - lse2) : 0.f;
-                        dsv[u] = p * (__uint_as_float(pv[e + u]) - dl);
+                        dsv[u] = p * dpm[16 * sc + e + u];
                     }
                     dk[8 * sc + e / 2] = pack_bf16x2(dsv[0], dsv[1]);
                 }
             }
-            tmem_st16(tmem + lane_base + kTmS + c0, dk);
+            tmem_st16(tmem + lane_base + s_buf + c0, dk);
             tmem_st_wait();
             tc_fence_before();
             __syncwarp();
