@@ -10,12 +10,13 @@
 //  1. delta_kernel: Delta per query row (one pass over O and dO).
 //  2. bwd_kernel, dK/dV CTAs (dkdv_body): one CTA per key tile (128 keys: 16 compacted
 //     8-row groups of the persistent slots, or a pair of local blocks); it loops over the
-//     query tiles that attend to those keys (all of them for persistent keys; for local
-//     blocks the query tiles whose query blocks selected either block).  S^T = K Q^T and
-//     dP^T = V dO^T land in TMEM (lanes = keys); 16 element warps (a key-row quarter and 32
-//     query columns each) form P^T and dS^T, write them as bf16 back over S^T / dP^T, and
-//     two TS MMAs accumulate dV += P^T dO and dK += dS^T Q in TMEM (dO and Q tiles read
-//     MN-major from shared memory).
+//     64-row query blocks that attend to those keys (all of them for persistent keys; for
+//     local blocks only the query blocks that selected either block).  S^T = K Q^T and
+//     dP^T = V dO^T (128 keys x 64 queries) land in one of two TMEM buffers (lanes = keys);
+//     16 element warps (a key-row quarter and 16 query columns each) form P^T and dS^T,
+//     write them as bf16 back over S^T / dP^T, and two TS MMAs accumulate dV += P^T dO and
+//     dK += dS^T Q in TMEM (dO and Q blocks read MN-major from shared memory).  The next
+//     query block's S^T / dP^T are computed while the current one is in the element warps.
 //  3. bwd_kernel, dQ CTAs (dq_body): one CTA per query tile (the forward's tiling); per key
 //     tile S = Q K^T and dP = dO V^T in TMEM, the element warps (a query-row quarter and 32
 //     key columns each) form dS, write it as bf16 over S, and a TS MMA accumulates
@@ -54,7 +55,6 @@ static_assert(kCw == 32, "column masks are 32-bit words");
 __host__ __device__ constexpr uint32_t packed_col(int kk) {
     return static_cast<uint32_t>(kCw * (kk / (kCw / 16)) + 8 * (kk % (kCw / 16)));
 }
-constexpr int kNst = 2;
 constexpr float kLog2e = 1.4426950408889634f;
 
 
@@ -142,26 +142,31 @@ __device__ __forceinline__ void zero_tiles(uint8_t* base, uint32_t bytes) {
     fence_proxy_async_smem();
 }
 
-constexpr int B_COUNT = 12;  // mbarrier slots reserved per CTA
+constexpr int B_COUNT = 16;  // mbarrier slots reserved per CTA
 
 // ===================================================================== dK / dV
+// A dK/dV CTA walks the query blocks that see its keys, one 64-row query block at a time:
+// Q and dO of a block are one TMA box each per 64 channels (16 KB for both halves of D),
+// kept in kQst stages with their lse / Delta.
+constexpr int kQst = 4;
+constexpr uint32_t kQBlk = 64 * 128;   // bytes of one query block, one 64-channel half
+
 struct DkdvPlan {
-    uint32_t k, v, q, dq_o, lse, dl, grp_row, qtl, qsel, bars, misc, total;
+    uint32_t k, v, q, dq_o, lse, dl, grp_row, sub, bars, misc, total;
 };
 
-__host__ __device__ inline DkdvPlan dkdv_plan(int D, int S, int n_qt) {
+__host__ __device__ inline DkdvPlan dkdv_plan(int D, int S, int qb_total) {
     DkdvPlan p;
     const uint32_t nh = D / 64;
     p.k = 0;
     p.v = p.k + nh * kHalf;
-    p.q = p.v + nh * kHalf;                 // kNst stages of Q
-    p.dq_o = p.q + kNst * nh * kHalf;       // kNst stages of dO
-    p.lse = p.dq_o + kNst * nh * kHalf;     // kNst x 128 fp32 (log2 units, +inf = padding)
-    p.dl = p.lse + kNst * 128 * 4;          // kNst x 128 fp32 Delta
-    p.grp_row = p.dl + kNst * 128 * 4;      // 8*S
-    p.qtl = p.grp_row + 4u * 8u * S;        // query tile list
-    p.qsel = p.qtl + 4u * n_qt;             // 4 selection bits per listed query tile
-    p.bars = (p.qsel + 4u * n_qt + 7u) & ~7u;
+    p.q = p.v + nh * kHalf;                 // kQst stages of one query block's Q
+    p.dq_o = p.q + kQst * nh * kQBlk;       // kQst stages of its dO
+    p.lse = p.dq_o + kQst * nh * kQBlk;     // kQst x 64 fp32 (log2 units, +inf = padding)
+    p.dl = p.lse + kQst * 64 * 4;           // kQst x 64 fp32 Delta
+    p.grp_row = p.dl + kQst * 64 * 4;       // 8*S
+    p.sub = p.grp_row + 4u * 8u * S;        // query blocks that see the keys: qb << 2 | bits
+    p.bars = (p.sub + 4u * qb_total + 7u) & ~7u;
     p.misc = p.bars + 8u * B_COUNT;
     p.total = p.misc + 4u * 8u;
     return p;
@@ -171,7 +176,6 @@ __host__ __device__ inline DkdvPlan dkdv_plan(int D, int S, int n_qt) {
 struct BwdKernelArgs {
     BwdArgs a;
     int n_pt_max;  // persistent key tiles per (b, h) of the dK/dV part
-    int n_qt;      // query tiles per (b, h)
     int ucap;      // capacity of a query tile's local-block union
     int n_dq_x;    // dQ CTAs per (b, h): query tiles
     int n_kd_x;    // dK/dV CTAs per (b, h): persistent + local key tiles
@@ -182,14 +186,18 @@ template <int D>
 __device__ __forceinline__ void dkdv_body(const BwdKernelArgs& ka, const int cta_x, const int h, const int b) {
     constexpr int NH = D / 64;
     constexpr uint32_t TILE = NH * kHalf;
-    constexpr uint32_t kTmS = 0, kTmP = 128, kTmDV = 256, kTmDK = 256 + D;
+    constexpr uint32_t QSTAGE = NH * kQBlk;
+    // TMEM: two buffers of (S^T | dP^T) for 64-query blocks (buffer x at 128 x, dP^T at +64),
+    // then the dV and dK accumulators
+    constexpr uint32_t kTmDV = 256, kTmDK = 256 + D;
     const BwdArgs& a = ka.a;
     const Geo& g = a.g;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
     const int S = g.S;
-    const DkdvPlan PL = dkdv_plan(D, S, ka.n_qt);
+    const int qb_total = a.q_frames / g.bt * g.nbf;
+    const DkdvPlan PL = dkdv_plan(D, S, qb_total);
     uint8_t* sK = sm + PL.k;
     uint8_t* sV = sm + PL.v;
     uint8_t* sQ = sm + PL.q;
@@ -197,15 +205,13 @@ __device__ __forceinline__ void dkdv_body(const BwdKernelArgs& ka, const int cta
     float* s_lse = reinterpret_cast<float*>(sm + PL.lse);
     float* s_dl = reinterpret_cast<float*>(sm + PL.dl);
     int32_t* grp_row = reinterpret_cast<int32_t*>(sm + PL.grp_row);
-    int32_t* qtl = reinterpret_cast<int32_t*>(sm + PL.qtl);
-    int32_t* qsel = reinterpret_cast<int32_t*>(sm + PL.qsel);
+    int32_t* sub = reinterpret_cast<int32_t*>(sm + PL.sub);
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + PL.bars);
     int* misc = reinterpret_cast<int*>(sm + PL.misc);
     volatile int* abort_flag = misc + 1;
 
     const int bh = b * g.H + h;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int qb_total = a.q_frames / g.bt * g.nbf;
     const int nq = a.q_frames * g.tf;
     const int nl = a.local_frames / g.bt * g.nbf;
     const uint32_t box_bytes = static_cast<uint32_t>(g.brows) * 128u;  // one block, one 64-channel half
@@ -213,20 +219,22 @@ __device__ __forceinline__ void dkdv_body(const BwdKernelArgs& ka, const int cta
     const int tile = pers_tile ? cta_x : cta_x - ka.n_pt_max;
 
     uint64_t* kv_full = &bars[0];      // K and V tiles of this CTA (once)
-    uint64_t* qd_full = &bars[1];      // [kNst] Q + dO + lse/Delta of a query tile
-    uint64_t* qd_empty = &bars[3];     // [kNst]
-    uint64_t* sdp_full = &bars[5];     // S^T and dP^T ready
-    uint64_t* pds_full = &bars[6];     // P^T and dS^T written (128 arrivals)
-    uint64_t* pass_done = &bars[7];    // dV/dK MMAs of a query tile done
-    uint64_t* drain = &bars[8];
+    uint64_t* qd_full = &bars[1];      // [kQst] Q + dO + lse/Delta of a query block
+    uint64_t* qd_empty = &bars[5];     // [kQst]
+    uint64_t* sdp_full = &bars[9];     // [2] S^T and dP^T of a query block in TMEM buffer x
+    uint64_t* pds_full = &bars[11];    // [2] P^T and dS^T written (one arrival per element warp)
+    uint64_t* pass_done = &bars[13];   // dV/dK MMAs of the last query block done (one phase)
+    uint64_t* drain = &bars[14];
     if (threadIdx.x == 0) {
         mbar_init(kv_full, 1);
-        for (int s = 0; s < kNst; ++s) {
+        for (int s = 0; s < kQst; ++s) {
             mbar_init(&qd_full[s], 1 + 32);  // producer expect_tx + 32 lse/Delta loaders
             mbar_init(&qd_empty[s], 1);
         }
-        mbar_init(sdp_full, 1);
-        mbar_init(pds_full, kElemWarps);  // one arrival per element warp
+        for (int x = 0; x < 2; ++x) {
+            mbar_init(&sdp_full[x], 1);
+            mbar_init(&pds_full[x], kElemWarps);
+        }
         mbar_init(pass_done, 1);
         mbar_init(drain, 1);
         misc[1] = 0;
@@ -248,43 +256,34 @@ __device__ __forceinline__ void dkdv_body(const BwdKernelArgs& ka, const int cta
     }
     __syncthreads();
     if (pers_tile) G = misc[2];
-    // the query tiles that see these keys, with selection bits
-    //   bit (2*kb + hq): key block kb (0/1) was selected by query block 2*qt + hq
+    // the query blocks that see these keys, in order, with bit kb set when the block selected
+    // key block kb (persistent keys: every query block, both bits)
     if (warp < 4) {
-        const int n_qt = ka.n_qt;
         int count = 0;
-        for (int t0 = 0; t0 < n_qt; t0 += 128) {
-            const int qt = t0 + threadIdx.x;
+        for (int q0 = 0; q0 < qb_total; q0 += 128) {
+            const int qb = q0 + threadIdx.x;
             int bits = 0;
-            if (qt < n_qt) {
+            if (qb < qb_total) {
                 if (pers_tile) {
-                    bits = 0xF;
+                    bits = 3;
                 } else {
-                    for (int hq = 0; hq < 2; ++hq) {
-                        const int qb = 2 * qt + hq;
-                        if (qb >= qb_total) continue;
-                        const int c = min(max(a.cnt[(size_t)bh * qb_total + qb], 0), a.idx_stride);
-                        const int32_t* row = a.idx + ((size_t)bh * qb_total + qb) * a.idx_stride;
-                        for (int i = 0; i < c; ++i) {
-                            const int v = row[i];
-                            if (v == L0) bits |= 1 << (0 + hq);
-                            if (L1 >= 0 && v == L1) bits |= 1 << (2 + hq);
-                        }
+                    const int c = min(max(a.cnt[(size_t)bh * qb_total + qb], 0), a.idx_stride);
+                    const int32_t* row = a.idx + ((size_t)bh * qb_total + qb) * a.idx_stride;
+                    for (int i = 0; i < c; ++i) {
+                        const int v = row[i];
+                        if (v == L0) bits |= 1;
+                        if (L1 >= 0 && v == L1) bits |= 2;
                     }
                 }
             }
-            // block-wide compaction of the tiles with bits != 0 (4 warps)
+            // block-wide compaction of the blocks with bits != 0 (4 warps)
             const unsigned m = __ballot_sync(0xffffffffu, bits != 0);
             __shared__ int wcount[4];
             if (lane == 0) wcount[warp] = __popc(m);
             named_bar_sync(1, 128);
             int base = count;
             for (int w = 0; w < warp; ++w) base += wcount[w];
-            if (bits) {
-                const int pos = base + __popc(m & ((1u << lane) - 1u));
-                qtl[pos] = qt;
-                qsel[pos] = bits;
-            }
+            if (bits) sub[base + __popc(m & ((1u << lane) - 1u))] = (qb << 2) | bits;
             count += wcount[0] + wcount[1] + wcount[2] + wcount[3];
             named_bar_sync(1, 128);
         }
@@ -294,7 +293,7 @@ __device__ __forceinline__ void dkdv_body(const BwdKernelArgs& ka, const int cta
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = static_cast<uint32_t>(misc[0]);
-    const int n_items = misc[3];
+    const int n_sub = misc[3];
     const bool live = pers_tile ? (tile * 16 < G) : true;
 
     if (live && warp == kProdWarp) {
@@ -319,117 +318,120 @@ __device__ __forceinline__ void dkdv_body(const BwdKernelArgs& ka, const int cta
             }
         }
         __syncwarp();
-        // in-block coordinates of this lane's four rows of a query tile (rows lane + 32 u:
-        // u = 0, 1 in its first query block, u = 2, 3 in its second); fixed for the CTA
-        int rt[4], ry[4], rx[4];
-        bool rin[4];
+        // in-block coordinates of this lane's two rows of a query block (rows lane, lane + 32)
+        int rt[2], ry[2], rx[2];
+        bool rin[2];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int rr = (lane + 32 * u) & 63;
-            rx[u] = rr % g.bw;
-            ry[u] = (rr / g.bw) % g.bh;
-            rt[u] = rr / (g.bw * g.bh);
-            rin[u] = rr < g.brows;
+        for (int v = 0; v < 2; ++v) {
+            const int rr = lane + 32 * v;
+            rx[v] = rr % g.bw;
+            ry[v] = (rr / g.bw) % g.bh;
+            rt[v] = rr / (g.bw * g.bh);
+            rin[v] = rr < g.brows;
         }
         int issued = 0;
-        for (int j = 0; j < n_items; ++j) {
-            const int st = j % kNst;
-            const int qt = qtl[j];
-            // lse (log2 units) and Delta of the tile's 128 query rows, read from global memory
-            // before waiting for the stage so that their latency overlaps the wait; +inf lse
-            // masks padding rows
-            float l2v[4], dlv[4];
+        for (int u = 0; u < n_sub; ++u) {
+            const int st = u % kQst;
+            const int qb = sub[u] >> 2;
+            // lse (log2 units) and Delta of the block's 64 rows, read from global memory before
+            // waiting for the stage so that their latency overlaps the wait; +inf lse masks
+            // rows outside the frame
+            const BlockBox qbb = block_box(g, qb % g.nbf);
+            const size_t base = (size_t)bh * nq + (size_t)(qb / g.nbf) * g.bt * g.tf + qbb.y0 * g.fw + qbb.x0;
+            float l2v[2], dlv[2];
 #pragma unroll
-            for (int hq = 0; hq < 2; ++hq) {
-                const int qb = 2 * qt + hq;
-                BlockBox qbb = {0, 0, 0, 0};
-                size_t base = 0;
-                if (qb < qb_total) {
-                    qbb = block_box(g, qb % g.nbf);
-                    base = (size_t)bh * nq + (size_t)(qb / g.nbf) * g.bt * g.tf + qbb.y0 * g.fw + qbb.x0;
-                }
-#pragma unroll
-                for (int v = 0; v < 2; ++v) {
-                    const int u = 2 * hq + v;
-                    l2v[u] = CUDART_INF_F;
-                    dlv[u] = 0.f;
-                    if (qb < qb_total && rin[u] && ry[u] < qbb.hv && rx[u] < qbb.wv) {
-                        const size_t t = base + (size_t)rt[u] * g.tf + ry[u] * g.fw + rx[u];
-                        l2v[u] = a.lse[t] * kLog2e;
-                        dlv[u] = a.delta[t];
-                    }
+            for (int v = 0; v < 2; ++v) {
+                l2v[v] = CUDART_INF_F;
+                dlv[v] = 0.f;
+                if (rin[v] && ry[v] < qbb.hv && rx[v] < qbb.wv) {
+                    const size_t t = base + (size_t)rt[v] * g.tf + ry[v] * g.fw + rx[v];
+                    l2v[v] = a.lse[t] * kLog2e;
+                    dlv[v] = a.delta[t];
                 }
             }
-            if (j >= kNst) {
-                const bool w = __all_sync(0xffffffffu, mbar_wait(&qd_empty[st], ((j / kNst) - 1) & 1, abort_flag, a.status));
+            if (u >= kQst) {
+                const bool w = __all_sync(0xffffffffu, mbar_wait(&qd_empty[st], ((u / kQst) - 1) & 1, abort_flag, a.status));
                 if (!w) break;
             }
             if (lane == 0) {
-                mbar_arrive_expect_tx(&qd_full[st], 2 * 2 * NH * box_bytes);
-                for (int hq = 0; hq < 2; ++hq) {
-                    const int qb = min(2 * qt + hq, qb_total - 1);
-                    const BlockBox qbb = block_box(g, qb % g.nbf);
-                    const int f0 = b * a.q_frames + (qb / g.nbf) * g.bt;
-                    for (int hh = 0; hh < NH; ++hh) {
-                        tma_load_5d(sQ + st * TILE + hh * kHalf + hq * (kHalf / 2), &a.tm_q, &qd_full[st],
-                                    hh * 64, h, qbb.x0, qbb.y0, f0);
-                        tma_load_5d(sDO + st * TILE + hh * kHalf + hq * (kHalf / 2), &a.tm_do, &qd_full[st],
-                                    hh * 64, h, qbb.x0, qbb.y0, f0);
-                    }
+                mbar_arrive_expect_tx(&qd_full[st], 2 * NH * box_bytes);
+                const int f0 = b * a.q_frames + (qb / g.nbf) * g.bt;
+                for (int hh = 0; hh < NH; ++hh) {
+                    tma_load_5d(sQ + st * QSTAGE + hh * kQBlk, &a.tm_q, &qd_full[st], hh * 64, h, qbb.x0, qbb.y0, f0);
+                    tma_load_5d(sDO + st * QSTAGE + hh * kQBlk, &a.tm_do, &qd_full[st], hh * 64, h, qbb.x0, qbb.y0, f0);
                 }
             }
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                s_lse[st * 128 + lane + 32 * u] = l2v[u];
-                s_dl[st * 128 + lane + 32 * u] = dlv[u];
+            for (int v = 0; v < 2; ++v) {
+                s_lse[st * 64 + lane + 32 * v] = l2v[v];
+                s_dl[st * 64 + lane + 32 * v] = dlv[v];
             }
             mbar_arrive(&qd_full[st]);
             ++issued;
         }
         if (lane == 0 && *abort_flag) {
             mbar_wait_drain(kv_full, 0, 100000000ull);
-            for (int j = max(0, issued - kNst); j < issued; ++j)
-                mbar_wait_drain(&qd_full[j % kNst], (j / kNst) & 1, 100000000ull);
+            for (int u = max(0, issued - kQst); u < issued; ++u)
+                mbar_wait_drain(&qd_full[u % kQst], (u / kQst) & 1, 100000000ull);
         }
     } else if (live && warp == kMmaWarp) {
         // ---------------------------------------------------------------- MMA
         if (lane == 0) {
-            constexpr uint32_t id_s = idesc_bf16(128, 128, false, false);
+            constexpr uint32_t id_s = idesc_bf16(128, 64, false, false);   // 128 keys x 64 queries
             constexpr uint32_t id_g = idesc_bf16(128, D, false, true);
             bool ok = mbar_wait(kv_full, 0, abort_flag, a.status);
             const uint32_t kb = smem_u32(sK), vb = smem_u32(sV);
-            for (int j = 0; ok && j < n_items; ++j) {
-                const int st = j % kNst;
-                if (!mbar_wait(&qd_full[st], (j / kNst) & 1, abort_flag, a.status)) { ok = false; break; }
-                // no wait for the previous tile's dV/dK MMAs: MMAs issued by this thread run in
-                // issue order, so they finish reading P^T/dS^T before S^T/dP^T overwrite them
+            // S^T = K Q_u^T and dP^T = V dO_u^T of query block u into TMEM buffer u & 1; the
+            // element warps turn them into P^T / dS^T (bf16, in place); dV += P^T dO_u and
+            // dK += dS^T Q_u follow.  Issue order: block u + 2's S^T / dP^T right after block u's
+            // dV / dK (the tensor pipe runs one thread's MMAs in issue order, so they never
+            // overwrite P^T / dS^T before dV / dK have read them), which keeps the next block's
+            // S^T / dP^T computing while the element warps work on the current one.
+            auto issue_sdp = [&](int u) -> bool {
+                const int st = u % kQst;
+                if (!mbar_wait(&qd_full[st], (u / kQst) & 1, abort_flag, a.status)) return false;
                 tc_fence_after();
-                const uint32_t qb_ = smem_u32(sQ + st * TILE), ob = smem_u32(sDO + st * TILE);
+                const uint32_t qs = smem_u32(sQ + st * QSTAGE), os = smem_u32(sDO + st * QSTAGE);
+                const uint32_t buf = tmem + 128 * (u & 1);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
-                    umma_ss(tmem + kTmS, sdesc_make(sdesc_lo(kb, 16) + (off >> 4)), sdesc_make(sdesc_lo(qb_, 16) + (off >> 4)), id_s, kk > 0);
+                    const uint32_t ka_ = (kk >> 2) * kHalf + (kk & 3) * 32;   // K / V tile: 128 rows
+                    const uint32_t kq = (kk >> 2) * kQBlk + (kk & 3) * 32;    // Q / dO block: 64 rows
+                    umma_ss(buf, sdesc_make(sdesc_lo(kb, 16) + (ka_ >> 4)), sdesc_make(sdesc_lo(qs, 16) + (kq >> 4)),
+                            id_s, kk > 0);
                 }
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
-                    umma_ss(tmem + kTmP, sdesc_make(sdesc_lo(vb, 16) + (off >> 4)), sdesc_make(sdesc_lo(ob, 16) + (off >> 4)), id_s, kk > 0);
+                    const uint32_t ka_ = (kk >> 2) * kHalf + (kk & 3) * 32;
+                    const uint32_t kq = (kk >> 2) * kQBlk + (kk & 3) * 32;
+                    umma_ss(buf + 64, sdesc_make(sdesc_lo(vb, 16) + (ka_ >> 4)), sdesc_make(sdesc_lo(os, 16) + (kq >> 4)),
+                            id_s, kk > 0);
                 }
-                umma_commit(sdp_full);
-                if (!mbar_wait(pds_full, j & 1, abort_flag, a.status)) { ok = false; break; }
+                umma_commit(&sdp_full[u & 1]);
+                return true;
+            };
+            for (int u = 0; ok && u < min(2, n_sub); ++u) ok = issue_sdp(u);
+            for (int u = 0; ok && u < n_sub; ++u) {
+                const int st = u % kQst;
+                if (!mbar_wait(&pds_full[u & 1], (u >> 1) & 1, abort_flag, a.status)) { ok = false; break; }
                 tc_fence_after();
+                const uint32_t qs = smem_u32(sQ + st * QSTAGE), os = smem_u32(sDO + st * QSTAGE);
+                const uint32_t buf = tmem + 128 * (u & 1);
+                // B operands dO / Q read MN-major: 64 channels per 128-byte row, the next 64
+                // channels kQBlk bytes on, 16 query rows per MMA
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    umma_ts(tmem + kTmDV, tmem + kTmS + packed_col(kk), sdesc_make(sdesc_lo(ob, kHalf) + kk * 128), id_g,
-                            (j > 0 || kk > 0) ? 1u : 0u);
-                }
+                for (int kk = 0; kk < 4; ++kk)
+                    umma_ts(tmem + kTmDV, buf + 16 * kk, sdesc_make(sdesc_lo(os, kQBlk) + kk * 128), id_g,
+                            (u > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    umma_ts(tmem + kTmDK, tmem + kTmP + packed_col(kk), sdesc_make(sdesc_lo(qb_, kHalf) + kk * 128), id_g,
-                            (j > 0 || kk > 0) ? 1u : 0u);
-                }
-                umma_commit(pass_done);
+                for (int kk = 0; kk < 4; ++kk)
+                    umma_ts(tmem + kTmDK, buf + 64 + 16 * kk, sdesc_make(sdesc_lo(qs, kQBlk) + kk * 128), id_g,
+                            (u > 0 || kk > 0) ? 1u : 0u);
                 umma_commit(&qd_empty[st]);
+                // one phase, after the last block: the element warps may run two blocks ahead of
+                // the dV/dK MMAs, so a per-block phase could not be waited on by parity alone
+                if (u == n_sub - 1) umma_commit(pass_done);
+                if (u + 2 < n_sub && !issue_sdp(u + 2)) { ok = false; break; }
             }
             if (!ok) {
                 umma_commit(drain);
@@ -439,12 +441,12 @@ __device__ __forceinline__ void dkdv_body(const BwdKernelArgs& ka, const int cta
     } else if (live && warp < kElemWarps) {
         // ------------------------------------------------------- element warps
         // warp w reads TMEM lanes 32 (w % 4).. (its key rows) and query columns
-        // [32 (w / 4), +32) of S^T / dP^T; it packs P^T / dS^T (bf16) into the first 16 of
-        // those columns once it has read them, so no other warp's input is overwritten.
+        // [16 (w / 4), +16) of the block's S^T / dP^T; it packs P^T / dS^T (bf16) into the
+        // first 8 of those columns once it has read them, so no other warp's input is
+        // overwritten.
         const int wq = warp & 3, cg = warp >> 2;
         const int r = 32 * wq + lane;
-        const int c0 = kCw * cg;            // first query column of this warp
-        const int hq = c0 >> 6;             // query block (half of the query tile) of those columns
+        const int c0 = 16 * cg;             // first query column of this warp
         const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
         const float sl2 = kLog2e / sqrtf(static_cast<float>(D));
         bool key_valid;
@@ -466,54 +468,54 @@ __device__ __forceinline__ void dkdv_body(const BwdKernelArgs& ka, const int cta
             return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, a.status));
         };
         bool ok = true;
-        for (int j = 0; j < n_items; ++j) {
-            const int st = j % kNst;
-            // lse/Delta of this query tile (written by the producer warp)
-            if (!wwait(&qd_full[st], (j / kNst) & 1)) { ok = false; break; }
-            if (!wwait(sdp_full, j & 1)) { ok = false; break; }
+        for (int u = 0; u < n_sub; ++u) {
+            const int st = u % kQst;
+            // lse/Delta of this query block (written by the producer warp)
+            if (!wwait(&qd_full[st], (u / kQst) & 1)) { ok = false; break; }
+            if (!wwait(&sdp_full[u & 1], (u >> 1) & 1)) { ok = false; break; }
             tc_fence_after();
-            const bool sel = key_valid && ((qsel[j] >> (2 * kbr + hq)) & 1);
-            const float l_mine = s_lse[st * 128 + c0 + lane];
-            const float d_mine = s_dl[st * 128 + c0 + lane];
-            uint32_t pk[kCw / 2], dk[kCw / 2];
-#pragma unroll
-            for (int sc = 0; sc < kCw / 16; ++sc) {
+            const bool sel = key_valid && ((sub[u] >> kbr) & 1);
+            const float l_mine = s_lse[st * 64 + c0 + (lane & 15)];
+            const float d_mine = s_dl[st * 64 + c0 + (lane & 15)];
+            const uint32_t buf = 128 * (u & 1);
+            uint32_t pk[8], dk[8];
+            {
                 uint32_t sv[16], pv[16];
-                tmem_ld16(tmem + lane_base + kTmS + c0 + 16 * sc, sv);
-                tmem_ld16(tmem + lane_base + kTmP + c0 + 16 * sc, pv);
+                tmem_ld16(tmem + lane_base + buf + c0, sv);
+                tmem_ld16(tmem + lane_base + buf + 64 + c0, pv);
                 tmem_ld_wait();
 #pragma unroll
                 for (int e4 = 0; e4 < 4; ++e4) {
                     float ls[4], ds[4];
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        ls[u] = __shfl_sync(0xffffffffu, l_mine, 16 * sc + 4 * e4 + u);
-                        ds[u] = __shfl_sync(0xffffffffu, d_mine, 16 * sc + 4 * e4 + u);
+                    for (int v = 0; v < 4; ++v) {
+                        ls[v] = __shfl_sync(0xffffffffu, l_mine, 4 * e4 + v);
+                        ds[v] = __shfl_sync(0xffffffffu, d_mine, 4 * e4 + v);
                     }
                     float p[4], d[4];
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
+                    for (int v = 0; v < 4; ++v) {
                         // p is exactly 0 off the selection; dP^T there is finite (key rows past
                         // a slot's length are finite), so dS^T is exactly 0 as well
-                        p[u] = sel ? fast_exp2(__uint_as_float(sv[4 * e4 + u]) * sl2 - ls[u]) : 0.f;
-                        d[u] = p[u] * (__uint_as_float(pv[4 * e4 + u]) - ds[u]);
+                        p[v] = sel ? fast_exp2(__uint_as_float(sv[4 * e4 + v]) * sl2 - ls[v]) : 0.f;
+                        d[v] = p[v] * (__uint_as_float(pv[4 * e4 + v]) - ds[v]);
                     }
-                    pk[8 * sc + 2 * e4] = pack_bf16x2(p[0], p[1]);
-                    pk[8 * sc + 2 * e4 + 1] = pack_bf16x2(p[2], p[3]);
-                    dk[8 * sc + 2 * e4] = pack_bf16x2(d[0], d[1]);
-                    dk[8 * sc + 2 * e4 + 1] = pack_bf16x2(d[2], d[3]);
+                    pk[2 * e4] = pack_bf16x2(p[0], p[1]);
+                    pk[2 * e4 + 1] = pack_bf16x2(p[2], p[3]);
+                    dk[2 * e4] = pack_bf16x2(d[0], d[1]);
+                    dk[2 * e4 + 1] = pack_bf16x2(d[2], d[3]);
                 }
             }
-            tmem_st16(tmem + lane_base + kTmS + c0, pk);
-            tmem_st16(tmem + lane_base + kTmP + c0, dk);
+            tmem_st8(tmem + lane_base + buf + c0, pk);
+            tmem_st8(tmem + lane_base + buf + 64 + c0, dk);
             tmem_st_wait();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(pds_full);
+            if (lane == 0) mbar_arrive(&pds_full[u & 1]);
         }
         ok = named_bar_and(2, 32 * kElemWarps, ok);
-        if (ok && n_items > 0) {
-            ok = named_bar_and(2, 32 * kElemWarps, wwait(pass_done, (n_items - 1) & 1));
+        if (ok && n_sub > 0) {
+            ok = named_bar_and(2, 32 * kElemWarps, wwait(pass_done, 0));
             tc_fence_after();
         }
         if (ok) {
@@ -541,7 +543,7 @@ __device__ __forceinline__ void dkdv_body(const BwdKernelArgs& ka, const int cta
             // channel chunks of 16: chunk c goes to element warp column group c % kNwq
             for (int c = cg; c < D / 16; c += kNwq) {
                 uint32_t v[16], w[16];
-                if (n_items > 0) {
+                if (n_sub > 0) {
                     tmem_ld16(tmem + lane_base + kTmDV + 16 * c, v);
                     tmem_ld16(tmem + lane_base + kTmDK + 16 * c, w);
                     tmem_ld_wait();
@@ -834,7 +836,10 @@ __device__ __forceinline__ void dq_body(const BwdKernelArgs& ka, const int tile,
                 for (int kk = 0; kk < 8; ++kk)
                     umma_ts(tmem + kTmQ, s_buf + packed_col(kk), sdesc_make(sdesc_lo(kb, kHalf) + kk * 128), id_g,
                             (it > 0 || kk > 0) ? 1u : 0u);
-                umma_commit(dq_done);
+                // one phase, after the last tile: the element warps may finish a tile before the
+                // previous tile's dQ MMAs are even issued, so a per-tile phase could not be waited
+                // on by parity alone
+                if (it == n_tiles - 1) umma_commit(dq_done);
                 umma_commit(&k_empty[st]);
             }
             if (!ok) {
@@ -920,7 +925,7 @@ __device__ __forceinline__ void dq_body(const BwdKernelArgs& ka, const int tile,
         }
         ok = named_bar_and(2, 32 * kElemWarps, ok);
         if (ok && n_tiles > 0) {
-            ok = named_bar_and(2, 32 * kElemWarps, wwait(dq_done, (n_tiles - 1) & 1));
+            ok = named_bar_and(2, 32 * kElemWarps, wwait(dq_done, 0));
             tc_fence_after();
         }
         if (ok) {
@@ -984,8 +989,7 @@ cudaError_t launch_k(K kernel, const A& args, dim3 grid, size_t smem, cudaStream
 }  // namespace
 
 size_t attn_bwd_smem_bytes(const Geo& g, int q_frames, int ucap) {
-    const int n_qt = (q_frames / g.bt * g.nbf + 1) / 2;
-    const size_t a = dkdv_plan(g.D, g.S, n_qt).total + 1024;
+    const size_t a = dkdv_plan(g.D, g.S, q_frames / g.bt * g.nbf).total + 1024;
     const size_t b = dq_plan(g.D, g.S, ucap, g.nbf).total + 1024;
     size_t m = a > b ? a : b;
     return m < 120 * 1024 ? 120 * 1024 : m;
@@ -1003,7 +1007,6 @@ cudaError_t launch_attn_bwd(const BwdArgs& a, cudaStream_t st) {
     BwdKernelArgs ka;
     ka.a = a;
     ka.n_pt_max = (g.S * 8 + 15) / 16;
-    ka.n_qt = (qb_total + 1) / 2;
     ka.ucap = a.ucap;
     ka.n_dq_x = (qb_total + 1) / 2;
     ka.n_kd_x = ka.n_pt_max + (a.local_frames / g.bt * g.nbf + 1) / 2;
