@@ -516,7 +516,6 @@ int pbsa_attn_bwd(const pbsa_config* cfg, const void* q, int q_frames, const voi
     a.local_frames = local_frames;
     a.ring_head = ring_head;
     a.idx_stride = idx_stride;
-    a.ucap = fwd_ucap(cfg, g, idx_stride);
     a.pers_len = pers_len;
     a.idx = idx;
     a.cnt = cnt;
@@ -530,7 +529,7 @@ int pbsa_attn_bwd(const pbsa_config* cfg, const void* q, int q_frames, const voi
     a.dk_local = dk_local;
     a.dv_local = dv_local;
     a.status = status;
-    if (pbsa::attn_bwd_smem_bytes(g, q_frames, a.ucap) > 227 * 1024)
+    if (pbsa::attn_bwd_smem_bytes(g, q_frames) > 227 * 1024)
         return fail(PBSA_ERR_UNSUPPORTED, "backward tables do not fit in shared memory");
     if ((rc = map_tokens(&a.tm_q, q, g, (long long)g.B * q_frames)) != PBSA_OK) return rc;
     if ((rc = map_tokens(&a.tm_do, dout, g, (long long)g.B * q_frames)) != PBSA_OK) return rc;

@@ -334,6 +334,14 @@ __device__ __forceinline__ void tma_load_groups16(uint8_t* dst, uint32_t half_by
     }
 }
 
+// Adds v to the four floats at p (16-byte aligned) in global memory (fp32 reduction, no
+// value returned).
+__device__ __forceinline__ void red_add_f32x4(float* p, float4 v) {
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(v.x), "f"(v.y), "f"(v.z),
+                 "f"(v.w)
+                 : "memory");
+}
+
 // ------------------------------------------------------------------------ numerics
 __device__ __forceinline__ float fast_exp2(float x) {
     float y;

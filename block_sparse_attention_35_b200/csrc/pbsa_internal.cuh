@@ -88,7 +88,6 @@ struct BwdArgs {
     Geo g;
     int q_frames, local_frames, ring_head;
     int idx_stride;
-    int ucap;            // capacity of the per-tile union of selections
     const int32_t* pers_len;
     const int32_t* idx;
     const int32_t* cnt;
@@ -96,7 +95,7 @@ struct BwdArgs {
     const __nv_bfloat16* out;
     const __nv_bfloat16* dout;
     float* delta;        // [B, H, Nq] workspace
-    float* dq;
+    float* dq;           // zeroed by the delta pass, then accumulated by the key tiles
     float* dk_pers;
     float* dv_pers;
     float* dk_local;
@@ -123,7 +122,7 @@ cudaError_t launch_attn_fwd(const FwdArgs& a, bool with_mass, cudaStream_t st);
 size_t attn_fwd_smem_bytes(const Geo& g, int ucap);
 
 cudaError_t launch_attn_bwd(const BwdArgs& a, cudaStream_t st);
-size_t attn_bwd_smem_bytes(const Geo& g, int q_frames, int ucap);
+size_t attn_bwd_smem_bytes(const Geo& g, int q_frames);
 
 cudaError_t launch_cache_update(const Geo& g, const __nv_bfloat16* k_local,
                                 const __nv_bfloat16* v_local, int local_frames, int ring_head,

@@ -279,7 +279,8 @@ PBSA_API int pbsa_attn_fwd(const pbsa_config* cfg, const void* q, int q_frames,
  * scores).  Inputs are the forward's inputs plus its out and lse.
  *
  *   dout      [B, q_frames*T_f, H, D] bf16
- *   dq        [B, q_frames*T_f, H, D] fp32 out (overwritten)
+ *   dq        [B, q_frames*T_f, H, D] fp32 out (overwritten; the key tiles' shares are summed
+ *             with fp32 reductions in no fixed order, so two runs agree to rounding)
  *   dk_pers, dv_pers  [B, H, S, 64, D] fp32 out; rows < pers_len overwritten, others
  *             untouched
  *   dk_local, dv_local  ring [B, W*T_f, H, D] fp32 out; tokens of the window's frames

@@ -184,10 +184,12 @@ def test_slot_rows_past_length_do_not_leak(cuda_dev):
         assert int(buf.status.item()) == 0
         outs.append((buf.out.clone(), buf.lse.clone(), buf.mass_pers.clone(), g["dq"].clone(),
                      g["dkl"].clone()))
-    # outputs, lse and gradients are deterministic; the masses are summed across CTAs with
-    # atomics in any order, so they agree to rounding
+    # outputs, lse and dK/dV are deterministic; the masses and dQ are summed across CTAs
+    # with fp32 reductions in any order, so they agree to rounding
     for i, (a, b) in enumerate(zip(*outs)):
         if i == 2:
             assert torch.allclose(a, b, rtol=1e-6, atol=0)
+        elif i == 3:
+            assert torch.allclose(a, b, rtol=1e-5, atol=1e-6)
         else:
             assert torch.equal(a, b)
