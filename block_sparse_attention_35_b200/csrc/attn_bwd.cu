@@ -13,13 +13,15 @@
 //     persistent keys; for local blocks the query blocks that selected either block).  Per
 //     query block u:
 //       S^T = K Q_u^T, dP^T = V dO_u^T     128 keys x 64 queries, into one of two TMEM buffers
-//       16 element warps                   P^T (bf16, back over S^T in TMEM) and dS^T (bf16,
-//                                          into a 128B-swizzled shared-memory tile)
-//       dV += P^T dO_u  (A from TMEM),  dK += dS^T Q_u,  dQ^T_u = K^T dS^T
-//                                          (dQ^T_u into the buffer's dP^T columns)
-//       4 dQ warps                         read dQ^T_u and add it into dQ in global memory
-//                                          (fp32 reductions; a query row's other key tiles
-//                                          add theirs, so dQ is summed in no fixed order)
+//       16 element warps                   P^T and dS^T (bf16, packed over S^T in TMEM; dS^T
+//                                          also into a 128B-swizzled shared-memory tile)
+//       dV += P^T dO_u, dK += dS^T Q_u     (A from TMEM)
+//       dQ^T_u = K^T dS^T                  (both from shared memory, into the buffer's dP^T
+//                                          columns)
+//       4 dQ warps                         read dQ^T_u, stage it as the query block's box and
+//                                          add it into dQ with TMA reductions (a query row's
+//                                          other key tiles add theirs, so dQ is summed in no
+//                                          fixed order)
 //     Every tensor-core product is computed once: five GEMMs per (key tile, query block).
 //     The next query block's S^T is computed while the element warps work on the current
 //     one, and its dP^T as soon as the dQ warps have read the current dQ^T.
@@ -146,7 +148,7 @@ constexpr uint32_t kDsBuf = 128 * 128;  // dS^T of one query block: 128 keys x 6
 constexpr int B_COUNT = 20;             // mbarrier slots reserved per CTA
 
 struct BwdPlan {
-    uint32_t k, v, q, dq_o, ds, lse, dl, grp_row, sub, bars, misc, dqs, dqt, total;
+    uint32_t k, v, q, dq_o, ds, lse, dl, grp_row, sub, bars, misc, dqs, total;
 };
 
 __host__ __device__ inline BwdPlan bwd_plan(int D, int S, int qb_total) {
@@ -163,9 +165,8 @@ __host__ __device__ inline BwdPlan bwd_plan(int D, int S, int qb_total) {
     p.sub = p.grp_row + 4u * 8u * S;        // query blocks that see the keys: qb << 2 | bits
     p.bars = (p.sub + 4u * qb_total + 7u) & ~7u;
     p.misc = p.bars + 8u * B_COUNT;
-    p.dqs = (p.misc + 4u * 8u + 15u) & ~15u;  // dQ staging: 64 query rows x D fp32
-    p.dqt = p.dqs + 64u * 4u * D;           // per dQ warp: tokens of the block's 64 rows
-    p.total = p.dqt + 4u * 64u * kDqWarps;
+    p.dqs = (p.misc + 4u * 8u + 1023u) & ~1023u;  // dQ staging: per 64 channels, 64 rows x 64 fp32
+    p.total = p.dqs + 64u * 4u * D;
     return p;
 }
 
@@ -438,11 +439,11 @@ __device__ __forceinline__ void key_tile_body(const BwdKernelArgs& ka, const int
                 for (int kk = 0; kk < 4; ++kk)
                     umma_ts(tmem + kTmDV, buf + 16 * kk, sdesc_make(sdesc_lo(os, kQBlk) + kk * 128), id_g,
                             (u > 0 || kk > 0) ? 1u : 0u);
-                // dK: A = dS^T K-major (a key per 128-byte row, 16 queries = 32 bytes per MMA)
+                // dK: A = dS^T, packed next to P^T in TMEM
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    umma_ss(tmem + kTmDK, sdesc_make(sdesc_lo(ds, 16) + 2 * kk),
-                            sdesc_make(sdesc_lo(qs, kQBlk) + kk * 128), id_g, (u > 0 || kk > 0) ? 1u : 0u);
+                    umma_ts(tmem + kTmDK, buf + 16 * kk + 8, sdesc_make(sdesc_lo(qs, kQBlk) + kk * 128), id_g,
+                            (u > 0 || kk > 0) ? 1u : 0u);
                 // dQ^T = K^T dS^T: A = the K tile read MN-major (channels along M, the next 64
                 // channels kHalf bytes on), B = dS^T read MN-major (queries along N); 16 keys
                 // (2 KB of rows) per MMA
@@ -470,10 +471,11 @@ __device__ __forceinline__ void key_tile_body(const BwdKernelArgs& ka, const int
     } else if (live && warp < kElemWarps) {
         // ------------------------------------------------------- element warps
         // warp w reads TMEM lanes 32 (w % 4).. (its key rows) and query columns
-        // [16 (w / 4), +16) of the block's S^T / dP^T; it packs P^T (bf16) into the first 8 of
-        // its S^T columns once it has read them (so no other warp's input is overwritten) and
-        // writes dS^T (bf16) into its key rows of the block's dS^T tile: row r holds the 64
-        // queries in 128 bytes, 16-byte chunk c stored at chunk c ^ (r % 8) (128-byte swizzle)
+        // [16 (w / 4), +16) of the block's S^T / dP^T; once it has read them it packs P^T and
+        // dS^T (bf16) into its own 16 S^T columns (P^T first, so no other warp's input is
+        // overwritten) and writes dS^T into its key rows of the block's dS^T tile in shared
+        // memory: row r holds the 64 queries in 128 bytes, 16-byte chunk c stored at chunk
+        // c ^ (r % 8) (128-byte swizzle)
         const int wq = warp & 3, cg = warp >> 2;
         const int r = 32 * wq + lane;
         const int c0 = 16 * cg;             // first query column of this warp
@@ -503,7 +505,7 @@ __device__ __forceinline__ void key_tile_body(const BwdKernelArgs& ka, const int
             // lse/Delta of this query block (written by the producer warp)
             if (!wwait(&qd_full[st], (u / kQst) & 1)) { ok = false; break; }
             if (!wwait(&sdp_full[u & 1], (u >> 1) & 1)) { ok = false; break; }
-            // the dS^T tile is free once the dK / dQ^T MMAs of block u - 1 are done
+            // the dS^T tile is free once the dQ^T MMAs of block u - 1 are done
             if (u >= 1 && !wwait(&dq_full[(u - 1) & 1], ((u - 1) >> 1) & 1)) { ok = false; break; }
             tc_fence_after();
             const bool sel = key_valid && ((sub[u] >> kbr) & 1);
@@ -539,6 +541,7 @@ __device__ __forceinline__ void key_tile_body(const BwdKernelArgs& ka, const int
                 }
             }
             tmem_st8(tmem + lane_base + buf + c0, pk);
+            tmem_st8(tmem + lane_base + buf + c0 + 8, dk);
             {
                 uint8_t* row = sDS + r * 128;
 #pragma unroll
@@ -606,73 +609,51 @@ __device__ __forceinline__ void key_tile_body(const BwdKernelArgs& ka, const int
     } else if (live && warp >= kDqWarp0) {
         // ---------------------------------------------------------------- dQ warps
         // warp w reads TMEM lanes 32 (w % 4).. = channels of dQ^T.  Per query block: read the
-        // 64 query columns 32 at a time into a [query][channel] staging tile in shared memory,
-        // release the columns, then add the tile's rows into dQ, 16 rows per warp, with one
-        // 16-byte reduction per lane and row (a 128-channel row per warp instruction)
+        // 64 query columns into registers and release them, write them into a staging tile
+        // laid out as the query block's TMA box (per 64 channels: 64 rows of 64 fp32), and let
+        // one thread add the tile into dQ with TMA reductions (one per 64 channels; rows
+        // outside the frame are skipped).
         const int wq = warp & 3, dw = warp - kDqWarp0;
         const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
         const int ch = 32 * wq + lane;
         const float isd = 1.0f / sqrtf(static_cast<float>(D));
-        float* stage = reinterpret_cast<float*>(sm + PL.dqs);          // [64][D]
-        int32_t* tokw = reinterpret_cast<int32_t*>(sm + PL.dqt) + 64 * dw;
-        // in-block coordinates of query rows lane and lane + 32
-        int rt[2], ry[2], rx[2];
-        bool rin[2];
-#pragma unroll
-        for (int v = 0; v < 2; ++v) {
-            const int rr = lane + 32 * v;
-            rx[v] = rr % g.bw;
-            ry[v] = (rr / g.bw) % g.bh;
-            rt[v] = rr / (g.bw * g.bh);
-            rin[v] = rr < g.brows;
-        }
-        float* dq_bh = a.dq + (size_t)b * nq * g.H * D + (size_t)h * D;
+        float* stage = reinterpret_cast<float*>(sm + PL.dqs);
+        float* my_col = stage + (ch >> 6) * (64 * 64) + (ch & 63);   // column ch of row 0
+        const bool issuer = dw == 0 && lane == 0;
         for (int u = 0; u < n_sub; ++u) {
-            // token of query rows lane and lane + 32 of this block (-1: not a frame token)
-            const int qb = sub[u] >> 2;
-            const BlockBox qbb = block_box(g, qb % g.nbf);
-            const int tbase = (qb / g.nbf) * g.bt * g.tf + qbb.y0 * g.fw + qbb.x0;
-#pragma unroll
-            for (int v = 0; v < 2; ++v)
-                tokw[lane + 32 * v] = (rin[v] && ry[v] < qbb.hv && rx[v] < qbb.wv)
-                                          ? tbase + rt[v] * g.tf + ry[v] * g.fw + rx[v] : -1;
-            if (!__all_sync(0xffffffffu, mbar_wait(&dq_full[u & 1], (u >> 1) & 1, abort_flag, a.status))) break;
+            const bool okw = __all_sync(0xffffffffu, mbar_wait(&dq_full[u & 1], (u >> 1) & 1, abort_flag, a.status));
+            // the four warps leave together if any wait gave up
+            if (!named_bar_and(3, 32 * kDqWarps, okw)) break;
             tc_fence_after();
             const uint32_t col = tmem + lane_base + 128 * (u & 1) + 64;
-#pragma unroll
-            for (int hv = 0; hv < 2; ++hv) {
-                uint32_t v[32];
-                tmem_ld32(col + 32 * hv, v);
-                tmem_ld_wait();
-                if (ch < D) {
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) stage[(32 * hv + j) * D + ch] = __uint_as_float(v[j]) * isd;
-                }
-            }
+            uint32_t v0[32], v1[32];
+            tmem_ld32(col, v0);
+            tmem_ld32(col + 32, v1);
+            tmem_ld_wait();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&dq_free[u & 1]);
+            // the previous block's reductions have read the staging tile
+            if (issuer) tma_store_wait_read();
             named_bar_sync(3, 32 * kDqWarps);
-            // rows 16 dw .. 16 dw + 15, four at a time
+            if (ch < D) {
 #pragma unroll
-            for (int i0 = 0; i0 < 16; i0 += 4) {
-                int t4[4];
-                float4 r4[4];
+                for (int j = 0; j < 32; ++j) my_col[j * 64] = __uint_as_float(v0[j]) * isd;
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int j = 16 * dw + i0 + i;
-                    t4[i] = tokw[j];
-                    r4[i] = 4 * lane < D ? *reinterpret_cast<const float4*>(stage + j * D + 4 * lane)
-                                         : make_float4(0.f, 0.f, 0.f, 0.f);
-                }
-                if (4 * lane < D) {
-#pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        if (t4[i] >= 0) red_add_f32x4(dq_bh + (size_t)t4[i] * g.H * D + 4 * lane, r4[i]);
-                }
+                for (int j = 0; j < 32; ++j) my_col[(32 + j) * 64] = __uint_as_float(v1[j]) * isd;
             }
+            fence_proxy_async_smem();
             named_bar_sync(3, 32 * kDqWarps);
+            if (issuer) {
+                const int qb = sub[u] >> 2;
+                const BlockBox qbb = block_box(g, qb % g.nbf);
+                const int f0 = b * a.q_frames + (qb / g.nbf) * g.bt;
+                for (int hh = 0; hh < NH; ++hh)
+                    tma_reduce_add_5d(&a.tm_dq, stage + hh * (64 * 64), hh * 64, h, qbb.x0, qbb.y0, f0);
+                tma_store_commit();
+            }
         }
+        if (issuer) tma_store_wait_all();
     }
     tc_fence_before();
     __syncthreads();

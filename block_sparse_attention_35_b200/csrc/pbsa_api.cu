@@ -199,6 +199,24 @@ int map_tokens(CUtensorMap* m, const void* ptr, const pbsa::Geo& g, long long fr
     return PBSA_OK;
 }
 
+// The same token layout as map_tokens for an fp32 tensor, unswizzled: one box is a block's
+// rows x 64 channels, 256 bytes per row (the backward adds dQ tiles through it).
+int map_tokens_f32(CUtensorMap* m, const void* ptr, const pbsa::Geo& g, long long frames) {
+    auto enc = encode_fn();
+    if (!enc) return fail(PBSA_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+    cuuint64_t dims[5] = {(cuuint64_t)g.D, (cuuint64_t)g.H, (cuuint64_t)g.fw, (cuuint64_t)g.fh,
+                          (cuuint64_t)frames};
+    cuuint64_t strides[4] = {(cuuint64_t)g.D * 4, (cuuint64_t)g.H * g.D * 4,
+                             (cuuint64_t)g.fw * g.H * g.D * 4, (cuuint64_t)g.fh * g.fw * g.H * g.D * 4};
+    cuuint32_t box[5] = {64, 1, (cuuint32_t)g.bw, (cuuint32_t)g.bh, (cuuint32_t)g.bt};
+    cuuint32_t es[5] = {1, 1, 1, 1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 5, const_cast<void*>(ptr), dims, strides, box, es,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(PBSA_ERR_CUDA, "cuTensorMapEncodeTiled (fp32 tokens) failed: %d", (int)r);
+    return PBSA_OK;
+}
+
 // [rows, D] bf16 tensor (persistent slots, 64 rows each), box [8, 64], 128-byte swizzle.
 int map_rows(CUtensorMap* m, const void* ptr, const pbsa::Geo& g, long long rows, int box_rows = 8) {
     auto enc = encode_fn();
@@ -533,6 +551,7 @@ int pbsa_attn_bwd(const pbsa_config* cfg, const void* q, int q_frames, const voi
         return fail(PBSA_ERR_UNSUPPORTED, "backward tables do not fit in shared memory");
     if ((rc = map_tokens(&a.tm_q, q, g, (long long)g.B * q_frames)) != PBSA_OK) return rc;
     if ((rc = map_tokens(&a.tm_do, dout, g, (long long)g.B * q_frames)) != PBSA_OK) return rc;
+    if ((rc = map_tokens_f32(&a.tm_dq, dq, g, (long long)g.B * q_frames)) != PBSA_OK) return rc;
     if ((rc = map_tokens(&a.tm_kl, k_local, g, (long long)g.B * g.W)) != PBSA_OK) return rc;
     if ((rc = map_tokens(&a.tm_vl, v_local, g, (long long)g.B * g.W)) != PBSA_OK) return rc;
     if ((rc = map_slots(&a.tm_kp, &a.tm_kp64, k_pers, k_local, g)) != PBSA_OK) return rc;

@@ -140,6 +140,22 @@ __device__ __forceinline__ void tma_store_5d(const CUtensorMap* map, const void*
         : "memory");
 }
 
+// Adds a shared-memory tile into global memory through a 5-D tensor map (element-wise add of
+// the map's type, performed by TMA; elements outside the tensor are skipped).
+__device__ __forceinline__ void tma_reduce_add_5d(const CUtensorMap* map, const void* src, int c0,
+                                                  int c1, int c2, int c3, int c4) {
+    asm volatile(
+        "cp.reduce.async.bulk.tensor.5d.global.shared::cta.add.tile.bulk_group"
+        " [%0, {%2, %3, %4, %5, %6}], [%1];" ::"l"(map),
+        "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4)
+        : "memory");
+}
+
+// Waits until every committed bulk group has finished reading its shared-memory source.
+__device__ __forceinline__ void tma_store_wait_read() {
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+
 __device__ __forceinline__ void tma_store_commit() {
     asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
@@ -332,14 +348,6 @@ __device__ __forceinline__ void tma_load_groups16(uint8_t* dst, uint32_t half_by
             c += 1;
         }
     }
-}
-
-// Adds v to the four floats at p (16-byte aligned) in global memory (fp32 reduction, no
-// value returned).
-__device__ __forceinline__ void red_add_f32x4(float* p, float4 v) {
-    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(v.x), "f"(v.y), "f"(v.z),
-                 "f"(v.w)
-                 : "memory");
 }
 
 // ------------------------------------------------------------------------ numerics

@@ -103,6 +103,7 @@ struct BwdArgs {
     int32_t* status;
     CUtensorMap tm_q, tm_do, tm_kl, tm_vl, tm_kp, tm_vp;
     CUtensorMap tm_kp64, tm_vp64;
+    CUtensorMap tm_dq;   // dq as fp32 [B*q_frames, fh, fw, H, D], box of one block x 64 channels
 };
 
 // Launchers (return a cudaError_t from the launch).
