@@ -379,7 +379,7 @@ def run_ours(args, ws, rank, local):
         bwd_avg = parts["bwd"]
         bwd_ach = (sum(bwd_flops) / len(bwd_flops)) / (bwd_avg * 1e-3) / 1e12
         if bwd_avg > fwd_avg:
-            dominant = {"kernel": "attn_bwd (delta + dQ/dK/dV grid)", "achieved": bwd_ach, "ms": bwd_avg}
+            dominant = {"kernel": "attn_bwd (delta + key-tile grid)", "achieved": bwd_ach, "ms": bwd_avg}
     traffic = None
     tfile = os.path.join(ROOT, "profiles", "traffic.json")
     if os.path.exists(tfile):
