@@ -288,7 +288,7 @@ __device__ __forceinline__ void key_tile_body(const BwdKernelArgs& ka, const int
             for (int w = 0; w < warp; ++w) base += wcount[w];
             if (bits) {
                 int pos = base + __popc(m & ((1u << lane) - 1u));
-                if (pers_tile) pos = (pos + qb_total - (tile * 7) % qb_total) % qb_total;
+                if (pers_tile) pos = (pos + qb_total - tile % qb_total) % qb_total;
                 sub[pos] = (qb << 2) | bits;
             }
             count += wcount[0] + wcount[1] + wcount[2] + wcount[3];
