@@ -23,8 +23,8 @@
 //                                          other key tiles add theirs, so dQ is summed in no
 //                                          fixed order)
 //     Every tensor-core product is computed once: five GEMMs per (key tile, query block).
-//     The next query block's S^T is computed while the element warps work on the current
-//     one, and its dP^T as soon as the dQ warps have read the current dQ^T.
+//     S^T of block u + 2 is computed while the element warps work on block u + 1, and its
+//     dP^T as soon as the dQ warps have read dQ^T of block u out of the same columns.
 // Warp roles: 0-15 element warps, 16 TMA producer, 17 MMA, 18-21 dQ warps (one per TMEM
 // lane quarter).  Persistent slots of any length 1..64 are streamed as ceil(len / 8) groups;
 // key rows of a partial last group past the slot's length are masked (P and dS exactly zero),
