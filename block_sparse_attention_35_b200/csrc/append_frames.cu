@@ -10,8 +10,8 @@
 //
 // append_kernel: one CTA per (block of the new frames, batch item).  Each thread owns 8
 // consecutive channels of a token's [H, D] row (a CTA moves whole 3 KB rows of all heads,
-// fully coalesced), streams the block's valid tokens with 16-byte loads (four rows of K
-// and V, eight loads, in flight), stores K and V to their destination and, for window
+// fully coalesced), streams the block's valid tokens with 16-byte loads (up to eight rows of
+// K and V in flight), stores K and V to their destination and, for window
 // blocks, sums K for the mean in the order pool_kernel does (so the means are identical).
 // HBM traffic per appended frame: its K and V read once and written once.
 #include <cuda_bf16.h>
@@ -41,7 +41,10 @@ struct AppendParams {
     int32_t* pers_src;
 };
 
-__global__ void __launch_bounds__(1024) append_kernel(AppendParams p) {
+// ROWS token rows in flight per thread: 8 when the CTA has at most 512 threads
+// (H*D <= 4096), else 4 so that 1024 threads fit in the register file.
+template <int ROWS>
+__global__ void __launch_bounds__(ROWS > 4 ? 512 : 1024) append_kernel(AppendParams p) {
     const Geo& g = p.g;
     const int j = blockIdx.x, b = blockIdx.y;
     const int hd = g.H * g.D;
@@ -67,7 +70,7 @@ __global__ void __launch_bounds__(1024) append_kernel(AppendParams p) {
     float acc[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-    constexpr int kRows = 4;   // token rows in flight per thread
+    constexpr int kRows = ROWS;
     for (int r0 = 0; r0 < n; r0 += kRows) {
         uint4 kv[kRows], vv[kRows];
         long long off[kRows];
@@ -131,7 +134,10 @@ cudaError_t launch_append(const Geo& g, const __nv_bfloat16* k_new, const __nv_b
     AppendParams p{g, k_new, v_new, n_frames, n_sink, sink_group0, ring_slot, k_local, v_local, kbar,
                    k_pers, v_pers, pers_len, pers_score, pers_src};
     const int threads = (g.H * g.D / 8 + 31) / 32 * 32;
-    append_kernel<<<dim3(nblk, g.B), threads, 0, st>>>(p);
+    if (threads <= 512)
+        append_kernel<8><<<dim3(nblk, g.B), threads, 0, st>>>(p);
+    else
+        append_kernel<4><<<dim3(nblk, g.B), threads, 0, st>>>(p);
     return cudaGetLastError();
 }
 

@@ -38,7 +38,10 @@ struct PoolParams {
     float* kbar;  // [B, H, Wg*NB, D], by physical ring frame group
 };
 
-__global__ void __launch_bounds__(1024) pool_kernel(PoolParams p) {
+// ROWS rows in flight per thread: 16 when the CTA has at most 512 threads (H*D <= 4096),
+// else 8 so that 1024 threads fit in the register file.
+template <int ROWS>
+__global__ void __launch_bounds__(ROWS > 8 ? 512 : 1024) pool_kernel(PoolParams p) {
     const Geo& g = p.g;
     const int qb_total = p.q_frames / g.bt * g.nbf;
     const int blk = blockIdx.x;
@@ -79,10 +82,11 @@ __global__ void __launch_bounds__(1024) pool_kernel(PoolParams p) {
     for (int e = 0; e < 8; ++e) acc[e] = 0.f;
 
     const __nv_bfloat16* base = src + frame * g.tf * (long long)hd + t * 8;
-    for (int r0 = 0; r0 < n; r0 += 8) {
-        uint4 v[8];
+    // rows are summed in order, as append_kernel does
+    for (int r0 = 0; r0 < n; r0 += ROWS) {
+        uint4 v[ROWS];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
+        for (int u = 0; u < ROWS; ++u) {
             const int r = r0 + u;
             if (r < n) {
                 const int t = r / plane, y = y0 + (r % plane) / wv, x = x0 + r % wv;
@@ -90,7 +94,7 @@ __global__ void __launch_bounds__(1024) pool_kernel(PoolParams p) {
             }
         }
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
+        for (int u = 0; u < ROWS; ++u) {
             if (r0 + u < n) {
                 const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&v[u]);
 #pragma unroll
@@ -241,7 +245,10 @@ cudaError_t launch_pool(const Geo& g, const __nv_bfloat16* q, int q_frames,
     const int nblk = (q_frames + k_frames) / g.bt * g.nbf;
     if (nblk == 0) return cudaSuccess;
     const int threads = (g.H * g.D / 8 + 31) / 32 * 32;
-    pool_kernel<<<dim3(nblk, g.B), threads, 0, st>>>(p);
+    if (threads <= 512)
+        pool_kernel<16><<<dim3(nblk, g.B), threads, 0, st>>>(p);
+    else
+        pool_kernel<8><<<dim3(nblk, g.B), threads, 0, st>>>(p);
     return cudaGetLastError();
 }
 
