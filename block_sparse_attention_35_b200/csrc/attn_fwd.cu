@@ -418,10 +418,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
             constexpr uint32_t idesc_qk = idesc_bf16(128, 128, false, false);
             constexpr uint32_t idesc_pv = idesc_bf16(128, D, false, true);
             bool ok = mbar_wait(&bars[B_Q], 0, abort_flag, a.status);
+            // per-side state, indexed only by the unrolled side loops (so it stays in registers)
             int pend[2] = {-1, -1};    // stream tile whose PV is still to be issued, per side
             int nqk[2] = {0, 0};       // QK MMAs issued per side
             int npv[2] = {0, 0};       // PV MMAs issued per side
-            int vrem[kNst] = {0, 0};   // PVs still to read each V stage
+            static_assert(kNst == 2, "two V stages");
+            int vrem0 = 0, vrem1 = 0;  // PVs still to read each V stage
             const int n_side[2] = {n_side0, n_side1};
             auto issue_pv = [&](int X) -> bool {
                 const int t = pend[X], st = t % kNst;
@@ -437,7 +439,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                             (npv[X] > 0 || kk > 0) ? 1u : 0u);
                 umma_commit(&bars[B_PV + X]);
                 ++npv[X];
-                if (--vrem[st] == 0) umma_commit(&bars[B_VE + st]);
+                const int left = st ? --vrem1 : --vrem0;
+                if (left == 0) umma_commit(&bars[B_VE + st]);
                 pend[X] = -1;
                 return true;
             };
@@ -447,6 +450,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                 int lj;
                 const int cons = tile_cons(t, n_pt, nla, nlb, has_b, &lj);
                 const uint32_t k_base = smem_u32(sK + st * KV_BYTES);
+#pragma unroll
                 for (int X = 0; X < 2; ++X) {
                     if (cons & (1 << X)) {
                         if (pend[X] >= 0 && !issue_pv(X)) { ok = false; break; }
@@ -469,10 +473,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                 }
                 if (!ok) break;
                 umma_commit(&bars[B_KE + st]);
-                vrem[st] = __popc(cons);
+                if (st) vrem1 = __popc(cons);
+                else vrem0 = __popc(cons);
             }
-            for (int X = 0; ok && X < 2; ++X)
-                if (pend[X] >= 0 && !issue_pv(X)) ok = false;
+#pragma unroll
+            for (int X = 0; X < 2; ++X)
+                if (ok && pend[X] >= 0 && !issue_pv(X)) ok = false;
             if (!ok) {
                 // wait for the MMAs already issued before TMEM is released
                 umma_commit(&bars[B_DRAIN]);
