@@ -383,16 +383,33 @@ __device__ __forceinline__ void key_tile_body(const BwdKernelArgs& ka, const int
         }
     } else if (live && warp == kMmaWarp) {
         // ---------------------------------------------------------------- MMA
-        if (lane == 0) {
+        // the whole warp runs this (operands are warp-uniform); one elected lane issues each
+        // MMA and commit
+        {
+            auto mma_ss = [&](uint32_t d, uint64_t a_, uint64_t b_, uint32_t id, uint32_t acc) {
+                if (elect_one()) umma_ss(d, a_, b_, id, acc);
+                __syncwarp();
+            };
+            auto mma_ts = [&](uint32_t d, uint32_t a_, uint64_t b_, uint32_t id, uint32_t acc) {
+                if (elect_one()) umma_ts(d, a_, b_, id, acc);
+                __syncwarp();
+            };
+            auto commit = [&](uint64_t* bar) {
+                if (elect_one()) umma_commit(bar);
+                __syncwarp();
+            };
+            auto wwait = [&](uint64_t* bar, uint32_t parity) -> bool {
+                return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, a.status));
+            };
             constexpr uint32_t id_s = idesc_bf16(128, 64, false, false);   // 128 keys x 64 queries
             constexpr uint32_t id_g = idesc_bf16(128, D, false, true);      // dV, dK: B = dO / Q MN-major
             constexpr uint32_t id_q = idesc_bf16(128, 64, true, true);      // dQ^T: A = K^T, B = dS^T MN-major
-            bool ok = mbar_wait(kv_full, 0, abort_flag, a.status);
+            bool ok = wwait(kv_full, 0);
             const uint32_t kb = smem_u32(sK), vb = smem_u32(sV);
             // S^T = K Q_u^T into TMEM buffer u & 1 (columns +0), dP^T = V dO_u^T (+64)
             auto issue_s = [&](int u) -> bool {
                 const int st = u % kQst;
-                if (!mbar_wait(&qd_full[st], (u / kQst) & 1, abort_flag, a.status)) return false;
+                if (!wwait(&qd_full[st], (u / kQst) & 1)) return false;
                 tc_fence_after();
                 const uint32_t qs = smem_u32(sQ + st * QSTAGE);
                 const uint32_t buf = tmem + 128 * (u & 1);
@@ -400,7 +417,7 @@ __device__ __forceinline__ void key_tile_body(const BwdKernelArgs& ka, const int
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t ka_ = (kk >> 2) * kHalf + (kk & 3) * 32;   // K tile: 128 rows
                     const uint32_t kq = (kk >> 2) * kQBlk + (kk & 3) * 32;    // Q block: 64 rows
-                    umma_ss(buf, sdesc_make(sdesc_lo(kb, 16) + (ka_ >> 4)), sdesc_make(sdesc_lo(qs, 16) + (kq >> 4)),
+                    mma_ss(buf, sdesc_make(sdesc_lo(kb, 16) + (ka_ >> 4)), sdesc_make(sdesc_lo(qs, 16) + (kq >> 4)),
                             id_s, kk > 0);
                 }
                 return true;
@@ -413,10 +430,10 @@ __device__ __forceinline__ void key_tile_body(const BwdKernelArgs& ka, const int
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t ka_ = (kk >> 2) * kHalf + (kk & 3) * 32;
                     const uint32_t kq = (kk >> 2) * kQBlk + (kk & 3) * 32;
-                    umma_ss(buf + 64, sdesc_make(sdesc_lo(vb, 16) + (ka_ >> 4)), sdesc_make(sdesc_lo(os, 16) + (kq >> 4)),
+                    mma_ss(buf + 64, sdesc_make(sdesc_lo(vb, 16) + (ka_ >> 4)), sdesc_make(sdesc_lo(os, 16) + (kq >> 4)),
                             id_s, kk > 0);
                 }
-                umma_commit(&sdp_full[u & 1]);
+                commit(&sdp_full[u & 1]);
             };
             for (int u = 0; ok && u < min(2, n_sub); ++u) {
                 ok = issue_s(u);
@@ -428,7 +445,7 @@ __device__ __forceinline__ void key_tile_body(const BwdKernelArgs& ka, const int
             // the dP^T columns, dP^T of u + 2.
             for (int u = 0; ok && u < n_sub; ++u) {
                 const int st = u % kQst;
-                if (!mbar_wait(&pds_full[u & 1], (u >> 1) & 1, abort_flag, a.status)) { ok = false; break; }
+                if (!wwait(&pds_full[u & 1], (u >> 1) & 1)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t qs = smem_u32(sQ + st * QSTAGE), os = smem_u32(sDO + st * QSTAGE);
                 const uint32_t ds = smem_u32(sDS);
@@ -437,34 +454,34 @@ __device__ __forceinline__ void key_tile_body(const BwdKernelArgs& ka, const int
                 // channels kQBlk bytes on, 16 query rows per MMA
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    umma_ts(tmem + kTmDV, buf + 16 * kk, sdesc_make(sdesc_lo(os, kQBlk) + kk * 128), id_g,
+                    mma_ts(tmem + kTmDV, buf + 16 * kk, sdesc_make(sdesc_lo(os, kQBlk) + kk * 128), id_g,
                             (u > 0 || kk > 0) ? 1u : 0u);
                 // dK: A = dS^T, packed next to P^T in TMEM
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    umma_ts(tmem + kTmDK, buf + 16 * kk + 8, sdesc_make(sdesc_lo(qs, kQBlk) + kk * 128), id_g,
+                    mma_ts(tmem + kTmDK, buf + 16 * kk + 8, sdesc_make(sdesc_lo(qs, kQBlk) + kk * 128), id_g,
                             (u > 0 || kk > 0) ? 1u : 0u);
                 // dQ^T = K^T dS^T: A = the K tile read MN-major (channels along M, the next 64
                 // channels kHalf bytes on), B = dS^T read MN-major (queries along N); 16 keys
                 // (2 KB of rows) per MMA
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    umma_ss(buf + 64, sdesc_make(sdesc_lo(kb, kHalf) + kk * 128),
+                    mma_ss(buf + 64, sdesc_make(sdesc_lo(kb, kHalf) + kk * 128),
                             sdesc_make(sdesc_lo(ds, kDsBuf) + kk * 128), id_q, kk > 0 ? 1u : 0u);
-                umma_commit(&qd_empty[st]);
-                umma_commit(&dq_full[u & 1]);
+                commit(&qd_empty[st]);
+                commit(&dq_full[u & 1]);
                 // one phase, after the last block: the element warps may run two blocks ahead of
                 // the dV/dK MMAs, so a per-block phase could not be waited on by parity alone
-                if (u == n_sub - 1) umma_commit(pass_done);
+                if (u == n_sub - 1) commit(pass_done);
                 if (u + 2 < n_sub) {
                     if (!issue_s(u + 2)) { ok = false; break; }
-                    if (!mbar_wait(&dq_free[u & 1], (u >> 1) & 1, abort_flag, a.status)) { ok = false; break; }
+                    if (!wwait(&dq_free[u & 1], (u >> 1) & 1)) { ok = false; break; }
                     tc_fence_after();
                     issue_dp(u + 2);
                 }
             }
             if (!ok) {
-                umma_commit(drain);
+                commit(drain);
                 mbar_wait_drain(drain, 0, 100000000ull);
             }
         }
