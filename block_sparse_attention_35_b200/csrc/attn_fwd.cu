@@ -414,10 +414,27 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         }
     } else if (warp == 10) {
         // ------------------------------------------------------------- MMA issuer
-        if (lane == 0) {
+        // the whole warp runs this (operands are warp-uniform); one elected lane issues each
+        // MMA and commit
+        {
+            auto mma_ss = [&](uint32_t d, uint64_t a_, uint64_t b_, uint32_t id, uint32_t acc) {
+                if (elect_one()) umma_ss(d, a_, b_, id, acc);
+                __syncwarp();
+            };
+            auto mma_ts = [&](uint32_t d, uint32_t a_, uint64_t b_, uint32_t id, uint32_t acc) {
+                if (elect_one()) umma_ts(d, a_, b_, id, acc);
+                __syncwarp();
+            };
+            auto commit = [&](uint64_t* bar) {
+                if (elect_one()) umma_commit(bar);
+                __syncwarp();
+            };
+            auto wwait = [&](uint64_t* bar, uint32_t parity) -> bool {
+                return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, a.status));
+            };
             constexpr uint32_t idesc_qk = idesc_bf16(128, 128, false, false);
             constexpr uint32_t idesc_pv = idesc_bf16(128, D, false, true);
-            bool ok = mbar_wait(&bars[B_Q], 0, abort_flag, a.status);
+            bool ok = wwait(&bars[B_Q], 0);
             // per-side state, indexed only by the unrolled side loops (so it stays in registers)
             int pend[2] = {-1, -1};    // stream tile whose PV is still to be issued, per side
             int nqk[2] = {0, 0};       // QK MMAs issued per side
@@ -427,26 +444,26 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
             const int n_side[2] = {n_side0, n_side1};
             auto issue_pv = [&](int X) -> bool {
                 const int t = pend[X], st = t % kNst;
-                if (!mbar_wait(&bars[B_PF + X], npv[X] & 1, abort_flag, a.status)) return false;
-                if (!mbar_wait(&bars[B_VF + st], (t / kNst) & 1, abort_flag, a.status)) return false;
+                if (!wwait(&bars[B_PF + X], npv[X] & 1)) return false;
+                if (!wwait(&bars[B_VF + st], (t / kNst) & 1)) return false;
                 tc_fence_after();
                 const uint32_t p_tmem = tmem + 128 * X;
                 const uint32_t o_tmem = tmem + 256 + 128 * X;
                 const uint32_t v_base = smem_u32(sV + st * KV_BYTES);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    umma_ts(o_tmem, p_tmem + kk * 8, sdesc_make(sdesc_lo(v_base, kHalf) + kk * 128), idesc_pv,
+                    mma_ts(o_tmem, p_tmem + kk * 8, sdesc_make(sdesc_lo(v_base, kHalf) + kk * 128), idesc_pv,
                             (npv[X] > 0 || kk > 0) ? 1u : 0u);
-                umma_commit(&bars[B_PV + X]);
+                commit(&bars[B_PV + X]);
                 ++npv[X];
                 const int left = st ? --vrem1 : --vrem0;
-                if (left == 0) umma_commit(&bars[B_VE + st]);
+                if (left == 0) commit(&bars[B_VE + st]);
                 pend[X] = -1;
                 return true;
             };
             for (int t = 0; ok && t < n_stream; ++t) {
                 const int st = t % kNst;
-                if (!mbar_wait(&bars[B_KF + st], (t / kNst) & 1, abort_flag, a.status)) { ok = false; break; }
+                if (!wwait(&bars[B_KF + st], (t / kNst) & 1)) { ok = false; break; }
                 int lj;
                 const int cons = tile_cons(t, n_pt, nla, nlb, has_b, &lj);
                 const uint32_t k_base = smem_u32(sK + st * KV_BYTES);
@@ -460,10 +477,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
 #pragma unroll
                         for (int kk = 0; kk < D / 16; ++kk) {
                             const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
-                            umma_ss(s_tmem, sdesc_make(sdesc_lo(q_base, 16) + (off >> 4)), sdesc_make(sdesc_lo(k_base, 16) + (off >> 4)),
+                            mma_ss(s_tmem, sdesc_make(sdesc_lo(q_base, 16) + (off >> 4)), sdesc_make(sdesc_lo(k_base, 16) + (off >> 4)),
                                     idesc_qk, kk > 0 ? 1u : 0u);
                         }
-                        umma_commit(&bars[B_SF + X]);
+                        commit(&bars[B_SF + X]);
                         ++nqk[X];
                         pend[X] = t;
                     } else if (pend[X] >= 0 && nqk[X] == n_side[X]) {
@@ -472,7 +489,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                     }
                 }
                 if (!ok) break;
-                umma_commit(&bars[B_KE + st]);
+                commit(&bars[B_KE + st]);
                 if (st) vrem1 = __popc(cons);
                 else vrem0 = __popc(cons);
             }
@@ -481,7 +498,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                 if (ok && pend[X] >= 0 && !issue_pv(X)) ok = false;
             if (!ok) {
                 // wait for the MMAs already issued before TMEM is released
-                umma_commit(&bars[B_DRAIN]);
+                commit(&bars[B_DRAIN]);
                 mbar_wait_drain(&bars[B_DRAIN], 0, 100000000ull);
             }
         }
