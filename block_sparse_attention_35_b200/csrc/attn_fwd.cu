@@ -354,7 +354,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsIo));
       if (warp == 8 || warp == 9) {
         // ------------------------------------------------- TMA producers (K+Q, V)
-        if (lane == 0) {
+        // the whole warp runs this; one elected lane issues each copy and barrier arrival
+        {
+            auto one = [&](auto&& f) {
+                if (elect_one()) f();
+                __syncwarp();
+            };
             const bool isK = warp == 8;
             const CUtensorMap* mp = isK ? &a.tm_kp : &a.tm_vp;
             const CUtensorMap* mp64 = isK ? &a.tm_kp64 : &a.tm_vp64;
@@ -362,12 +367,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
             uint8_t* base = isK ? sK : sV;
             uint64_t* full = &bars[isK ? B_KF : B_VF];
             uint64_t* empty = &bars[isK ? B_KE : B_VE];
-            tma_prefetch_desc(mp);
-            tma_prefetch_desc(mp64);
-            tma_prefetch_desc(ml);
+            one([&] {
+                tma_prefetch_desc(mp);
+                tma_prefetch_desc(mp64);
+                tma_prefetch_desc(ml);
+            });
             if (isK) {
-                tma_prefetch_desc(&a.tm_q);
-                mbar_arrive_expect_tx(&bars[B_Q], 2 * 2 * NH * box_bytes);
+                one([&] {
+                    tma_prefetch_desc(&a.tm_q);
+                    mbar_arrive_expect_tx(&bars[B_Q], 2 * 2 * NH * box_bytes);
+                });
                 for (int X = 0; X < 2; ++X)
                     for (int hb = 0; hb < 2; ++hb) {
                         int qb = qblock(X, hb);
@@ -375,22 +384,26 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                         const BlockBox qbb = block_box(g, qb % g.nbf);
                         const int f0 = b * a.q_frames + (qb / g.nbf) * g.bt;
                         for (int hh = 0; hh < NH; ++hh)
-                            tma_load_5d(sQ + X * Q_SIDE + hh * kHalf + hb * (kHalf / 2), &a.tm_q, &bars[B_Q],
-                                        hh * 64, h, qbb.x0, qbb.y0, f0);
+                            one([&] {
+                                tma_load_5d(sQ + X * Q_SIDE + hh * kHalf + hb * (kHalf / 2), &a.tm_q, &bars[B_Q],
+                                            hh * 64, h, qbb.x0, qbb.y0, f0);
+                            });
                     }
             }
             int issued = 0;
             for (int t = 0; t < n_stream; ++t) {
                 const int st = t % kNst;
-                if (t >= kNst && !mbar_wait(&empty[st], ((t / kNst) - 1) & 1, abort_flag, a.status)) break;
+                if (t >= kNst &&
+                    !__all_sync(0xffffffffu, mbar_wait(&empty[st], ((t / kNst) - 1) & 1, abort_flag, a.status)))
+                    break;
                 uint8_t* dst = base + st * KV_BYTES;
                 int lj;
                 const int cons = tile_cons(t, n_pt, nla, nlb, has_b, &lj);
                 if (lj < 0) {
-                    mbar_arrive_expect_tx(&full[st], KV_BYTES);
-                    tma_load_groups16<NH>(dst, kHalf, mp, mp64, grp_row, t * 16, G, &full[st]);
+                    one([&] { mbar_arrive_expect_tx(&full[st], KV_BYTES); });
+                    tma_load_groups16_warp<NH>(dst, kHalf, mp, mp64, grp_row, t * 16, G, &full[st]);
                 } else {
-                    mbar_arrive_expect_tx(&full[st], 2 * NH * box_bytes);
+                    one([&] { mbar_arrive_expect_tx(&full[st], 2 * NH * box_bytes); });
                     const int X = cons == 2 ? 1 : 0;
                     const int U = X ? UB : UA;
                     for (int hb = 0; hb < 2; ++hb) {
@@ -399,13 +412,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                         // first ring frame of the block's group (groups never wrap the ring)
                         const int cf = b * g.W + (a.ring_head + (L / g.nbf) * g.bt) % g.W;
                         for (int hh = 0; hh < NH; ++hh)
-                            tma_load_5d(dst + hh * kHalf + hb * (kHalf / 2), ml, &full[st], hh * 64, h,
-                                        kbb.x0, kbb.y0, cf);
+                            one([&] {
+                                tma_load_5d(dst + hh * kHalf + hb * (kHalf / 2), ml, &full[st], hh * 64, h,
+                                            kbb.x0, kbb.y0, cf);
+                            });
                     }
                 }
                 ++issued;
             }
-            if (*abort_flag) {
+            if (lane == 0 && *abort_flag) {
                 // let the copies already issued land before the CTA leaves
                 if (isK) mbar_wait_drain(&bars[B_Q], 0, 100000000ull);
                 for (int t = max(0, issued - kNst); t < issued; ++t)

@@ -363,6 +363,26 @@ __device__ __forceinline__ void tma_load_groups16(uint8_t* dst, uint32_t half_by
     }
 }
 
+// tma_load_groups16 for a converged warp: every lane walks the (warp-uniform) group table,
+// one elected lane issues each copy.
+template <int NH>
+__device__ __forceinline__ void tma_load_groups16_warp(uint8_t* dst, uint32_t half_bytes, const CUtensorMap* m8,
+                                                       const CUtensorMap* m64, const int32_t* grp_row,
+                                                       int first, int G, uint64_t* bar) {
+    int c = 0;
+    while (c < 16) {
+        const int gi = first + c;
+        const int row = grp_row[gi < G ? gi : G - 1] & ~7;
+        const bool run8 = (c & 7) == 0 && gi + 7 < G && (grp_row[gi + 7] & ~7) == row + 56;
+#pragma unroll
+        for (int hh = 0; hh < NH; ++hh) {
+            if (elect_one()) tma_load_2d(dst + hh * half_bytes + c * 1024, run8 ? m64 : m8, bar, hh * 64, row);
+            __syncwarp();
+        }
+        c += run8 ? 8 : 1;
+    }
+}
+
 // ------------------------------------------------------------------------ numerics
 __device__ __forceinline__ float fast_exp2(float x) {
     float y;
