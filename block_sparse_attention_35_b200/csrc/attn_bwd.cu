@@ -360,13 +360,18 @@ __device__ __forceinline__ void key_tile_body(const BwdKernelArgs& ka, const int
                 const bool w = __all_sync(0xffffffffu, mbar_wait(&qd_empty[st], ((u / kQst) - 1) & 1, abort_flag, a.status));
                 if (!w) break;
             }
-            if (lane == 0) {
-                mbar_arrive_expect_tx(&qd_full[st], 2 * NH * box_bytes);
-                const int f0 = b * a.q_frames + (qb / g.nbf) * g.bt;
-                for (int hh = 0; hh < NH; ++hh) {
+            // copies issued by one elected lane of the converged warp
+            const int f0 = b * a.q_frames + (qb / g.nbf) * g.bt;
+            if (elect_one()) mbar_arrive_expect_tx(&qd_full[st], 2 * NH * box_bytes);
+            __syncwarp();
+#pragma unroll
+            for (int hh = 0; hh < NH; ++hh) {
+                if (elect_one())
                     tma_load_5d(sQ + st * QSTAGE + hh * kQBlk, &a.tm_q, &qd_full[st], hh * 64, h, qbb.x0, qbb.y0, f0);
+                __syncwarp();
+                if (elect_one())
                     tma_load_5d(sDO + st * QSTAGE + hh * kQBlk, &a.tm_do, &qd_full[st], hh * 64, h, qbb.x0, qbb.y0, f0);
-                }
+                __syncwarp();
             }
 #pragma unroll
             for (int v = 0; v < 2; ++v) {
