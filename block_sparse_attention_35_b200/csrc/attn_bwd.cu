@@ -444,7 +444,7 @@ __device__ __forceinline__ void key_tile_body(const BwdKernelArgs& ka, const int
                 ok = issue_s(u);
                 if (ok) issue_dp(u);
             }
-            // Per query block u: dV, dK and dQ^T of u, then S^T of u + 2 into the same buffer
+            // Per query block u: dQ^T, dV and dK of u, then S^T of u + 2 into the same buffer
             // (it overwrites P^T(u) only after dV(u) has read it: the tensor pipe runs one
             // thread's MMAs in issue order), then, once the dQ warps have read dQ^T(u) out of
             // the dP^T columns, dP^T of u + 2.
@@ -455,6 +455,15 @@ __device__ __forceinline__ void key_tile_body(const BwdKernelArgs& ka, const int
                 const uint32_t qs = smem_u32(sQ + st * QSTAGE), os = smem_u32(sDO + st * QSTAGE);
                 const uint32_t ds = smem_u32(sDS);
                 const uint32_t buf = tmem + 128 * (u & 1);
+                // dQ^T = K^T dS^T: A = the K tile read MN-major (channels along M, the next 64
+                // channels kHalf bytes on), B = dS^T read MN-major (queries along N); 16 keys
+                // (2 KB of rows) per MMA
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_ss(buf + 64, sdesc_make(sdesc_lo(kb, kHalf) + kk * 128),
+                            sdesc_make(sdesc_lo(ds, kDsBuf) + kk * 128), id_q, kk > 0 ? 1u : 0u);
+                // dQ^T first: its commit frees the dS^T tile for the next block's element warps
+                commit(&dq_full[u & 1]);
                 // B operands dO / Q read MN-major: 64 channels per 128-byte row, the next 64
                 // channels kQBlk bytes on, 16 query rows per MMA
 #pragma unroll
@@ -466,15 +475,7 @@ __device__ __forceinline__ void key_tile_body(const BwdKernelArgs& ka, const int
                 for (int kk = 0; kk < 4; ++kk)
                     mma_ts(tmem + kTmDK, buf + 16 * kk + 8, sdesc_make(sdesc_lo(qs, kQBlk) + kk * 128), id_g,
                             (u > 0 || kk > 0) ? 1u : 0u);
-                // dQ^T = K^T dS^T: A = the K tile read MN-major (channels along M, the next 64
-                // channels kHalf bytes on), B = dS^T read MN-major (queries along N); 16 keys
-                // (2 KB of rows) per MMA
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_ss(buf + 64, sdesc_make(sdesc_lo(kb, kHalf) + kk * 128),
-                            sdesc_make(sdesc_lo(ds, kDsBuf) + kk * 128), id_q, kk > 0 ? 1u : 0u);
                 commit(&qd_empty[st]);
-                commit(&dq_full[u & 1]);
                 // one phase, after the last block: the element warps may run two blocks ahead of
                 // the dV/dK MMAs, so a per-block phase could not be waited on by parity alone
                 if (u == n_sub - 1) commit(pass_done);
