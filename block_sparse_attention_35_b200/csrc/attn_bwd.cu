@@ -532,8 +532,10 @@ __device__ __forceinline__ void key_tile_body(const BwdKernelArgs& ka, const int
             if (u >= 1 && !wwait(&dq_full[(u - 1) & 1], ((u - 1) >> 1) & 1)) { ok = false; break; }
             tc_fence_after();
             const bool sel = key_valid && ((sub[u] >> kbr) & 1);
-            const float l_mine = s_lse[st * 64 + c0 + (lane & 15)];
-            const float d_mine = s_dl[st * 64 + c0 + (lane & 15)];
+            // lse and Delta of the warp's 16 query columns: broadcast 16-byte loads (every lane
+            // reads the same four columns)
+            const float4* lse4 = reinterpret_cast<const float4*>(s_lse + st * 64 + c0);
+            const float4* dl4 = reinterpret_cast<const float4*>(s_dl + st * 64 + c0);
             const uint32_t buf = 128 * (u & 1);
             uint32_t pk[8], dk[8];
             {
@@ -543,12 +545,9 @@ __device__ __forceinline__ void key_tile_body(const BwdKernelArgs& ka, const int
                 tmem_ld_wait();
 #pragma unroll
                 for (int e4 = 0; e4 < 4; ++e4) {
-                    float ls[4], ds[4];
-#pragma unroll
-                    for (int v = 0; v < 4; ++v) {
-                        ls[v] = __shfl_sync(0xffffffffu, l_mine, 4 * e4 + v);
-                        ds[v] = __shfl_sync(0xffffffffu, d_mine, 4 * e4 + v);
-                    }
+                    const float4 l4 = lse4[e4], d4 = dl4[e4];
+                    const float ls[4] = {l4.x, l4.y, l4.z, l4.w};
+                    const float ds[4] = {d4.x, d4.y, d4.z, d4.w};
                     float p[4], d[4];
 #pragma unroll
                     for (int v = 0; v < 4; ++v) {
