@@ -13,7 +13,7 @@
 //     persistent keys; for local blocks the query blocks that selected either block).  Per
 //     query block u:
 //       S^T = K Q_u^T, dP^T = V dO_u^T     128 keys x 64 queries, into one of two TMEM buffers
-//       16 element warps                   P^T and dS^T (bf16, packed over S^T in TMEM; dS^T
+//       8 element warps                    P^T and dS^T (bf16, packed over S^T in TMEM; dS^T
 //                                          also into a 128B-swizzled shared-memory tile)
 //       dV += P^T dO_u, dK += dS^T Q_u     (A from TMEM)
 //       dQ^T_u = K^T dS^T                  (both from shared memory, into the buffer's dP^T
@@ -25,7 +25,7 @@
 //     Every tensor-core product is computed once: five GEMMs per (key tile, query block).
 //     S^T of block u + 2 is computed while the element warps work on block u + 1, and its
 //     dP^T as soon as the dQ warps have read dQ^T of block u out of the same columns.
-// Warp roles: 0-15 element warps, 16 TMA producer, 17 MMA, 18-21 dQ warps (one per TMEM
+// Warp roles: 0-7 element warps, 8 TMA producer, 9 MMA, 10-13 dQ warps (one per TMEM
 // lane quarter).  Persistent slots of any length 1..64 are streamed as ceil(len / 8) groups;
 // key rows of a partial last group past the slot's length are masked (P and dS exactly zero),
 // so they only need to hold finite values.
@@ -40,9 +40,21 @@ namespace pbsa {
 namespace {
 
 constexpr uint32_t kHalf = 128 * 128;   // 128 rows x 64 bf16 channels
-// Warp roles: 16 element warps (four per TMEM lane quarter, each over 16 query columns),
+// Warp roles: 8 element warps (two per TMEM lane quarter, each over 32 query columns),
 // one TMA producer warp, one MMA warp, four dQ warps.
-constexpr int kElemWarps = 16;
+constexpr int kElemWarps = 8;
+constexpr int kColsW = 256 / kElemWarps;  // query columns per element warp (64 per block)
+static_assert(kColsW % 16 == 0 && kColsW * (kElemWarps / 4) == 64, "element warp columns");
+
+// tcgen05.ld of N (16 or 32) consecutive columns of the warp's lane quarter
+template <int N>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[N]) {
+    static_assert(N == 16 || N == 32, "16 or 32 columns");
+    if constexpr (N == 32)
+        tmem_ld32(taddr, r);
+    else
+        tmem_ld16(taddr, r);
+}
 constexpr int kProdWarp = kElemWarps;
 constexpr int kMmaWarp = kElemWarps + 1;
 constexpr int kDqWarp0 = kElemWarps + 2;
@@ -494,14 +506,15 @@ __device__ __forceinline__ void key_tile_body(const BwdKernelArgs& ka, const int
     } else if (live && warp < kElemWarps) {
         // ------------------------------------------------------- element warps
         // warp w reads TMEM lanes 32 (w % 4).. (its key rows) and query columns
-        // [16 (w / 4), +16) of the block's S^T / dP^T; once it has read them it packs P^T and
-        // dS^T (bf16) into its own 16 S^T columns (P^T first, so no other warp's input is
-        // overwritten) and writes dS^T into its key rows of the block's dS^T tile in shared
+        // [kColsW (w / 4), +kColsW) of the block's S^T / dP^T; once it has read them it packs
+        // P^T and dS^T (bf16) into its own S^T columns (per 16 queries: P^T into the first 8,
+        // dS^T into the next 8; no other warp's input is overwritten) and writes dS^T into its
+        // key rows of the block's dS^T tile in shared
         // memory: row r holds the 64 queries in 128 bytes, 16-byte chunk c stored at chunk
         // c ^ (r % 8) (128-byte swizzle)
         const int wq = warp & 3, cg = warp >> 2;
         const int r = 32 * wq + lane;
-        const int c0 = 16 * cg;             // first query column of this warp
+        const int c0 = kColsW * cg;         // first query column of this warp
         const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
         const float sl2 = kLog2e / sqrtf(static_cast<float>(D));
         bool key_valid;
@@ -537,14 +550,14 @@ __device__ __forceinline__ void key_tile_body(const BwdKernelArgs& ka, const int
             const float4* lse4 = reinterpret_cast<const float4*>(s_lse + st * 64 + c0);
             const float4* dl4 = reinterpret_cast<const float4*>(s_dl + st * 64 + c0);
             const uint32_t buf = 128 * (u & 1);
-            uint32_t pk[8], dk[8];
+            uint32_t pk[kColsW / 2], dk[kColsW / 2];
             {
-                uint32_t sv[16], pv[16];
-                tmem_ld16(tmem + lane_base + buf + c0, sv);
-                tmem_ld16(tmem + lane_base + buf + 64 + c0, pv);
+                uint32_t sv[kColsW], pv[kColsW];
+                tmem_ld_cols(tmem + lane_base + buf + c0, sv);
+                tmem_ld_cols(tmem + lane_base + buf + 64 + c0, pv);
                 tmem_ld_wait();
 #pragma unroll
-                for (int e4 = 0; e4 < 4; ++e4) {
+                for (int e4 = 0; e4 < kColsW / 4; ++e4) {
                     const float4 l4 = lse4[e4], d4 = dl4[e4];
                     const float ls[4] = {l4.x, l4.y, l4.z, l4.w};
                     const float ds[4] = {d4.x, d4.y, d4.z, d4.w};
@@ -562,12 +575,23 @@ __device__ __forceinline__ void key_tile_body(const BwdKernelArgs& ka, const int
                     dk[2 * e4 + 1] = pack_bf16x2(d[2], d[3]);
                 }
             }
-            tmem_st8(tmem + lane_base + buf + c0, pk);
-            tmem_st8(tmem + lane_base + buf + c0 + 8, dk);
+            // per 16 query columns: P^T packed into the first 8 of their S^T columns, dS^T
+            // into the next 8 (the layout the dV and dK MMAs read)
+#pragma unroll
+            for (int j = 0; j < kColsW / 16; ++j) {
+                uint32_t p8[8], d8[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    p8[e] = pk[8 * j + e];
+                    d8[e] = dk[8 * j + e];
+                }
+                tmem_st8(tmem + lane_base + buf + c0 + 16 * j, p8);
+                tmem_st8(tmem + lane_base + buf + c0 + 16 * j + 8, d8);
+            }
             {
                 uint8_t* row = sDS + r * 128;
 #pragma unroll
-                for (int j = 0; j < 2; ++j)
+                for (int j = 0; j < kColsW / 8; ++j)
                     *reinterpret_cast<uint4*>(row + ((((c0 >> 3) + j) ^ (r & 7)) << 4)) =
                         make_uint4(dk[4 * j], dk[4 * j + 1], dk[4 * j + 2], dk[4 * j + 3]);
             }
@@ -604,8 +628,8 @@ __device__ __forceinline__ void key_tile_body(const BwdKernelArgs& ka, const int
                 }
             }
             const float isd = 1.0f / sqrtf(static_cast<float>(D));
-            // channel chunks of 16: chunk c goes to element warp column group c % 4
-            for (int c = cg; c < D / 16; c += 4) {
+            // channel chunks of 16: chunk c goes to element warp column group c % (warps / 4)
+            for (int c = cg; c < D / 16; c += kElemWarps / 4) {
                 uint32_t v[16], w[16];
                 if (n_sub > 0) {
                     tmem_ld16(tmem + lane_base + kTmDV + 16 * c, v);

@@ -51,9 +51,9 @@ constexpr uint32_t kTmCols = 512;
 constexpr int kThreads = 384;
 // Register split: the kernel launches at kLaunchRegs per thread (384 x 168 = 64512); the
 // producer/MMA warpgroup drops to kRegsIo and both softmax warpgroups rise to kRegsSoftmax,
-// 2 x 128 x 200 + 128 x 104 = 64512, exactly the launch pool.  The host refuses to launch if
+// 2 x 128 x 216 + 128 x 72 = 64512, exactly the launch pool.  The host refuses to launch if
 // ptxas did not give the kernel kLaunchRegs, so the increase can always be satisfied.
-constexpr int kLaunchRegs = 168, kRegsIo = 104, kRegsSoftmax = 200;
+constexpr int kLaunchRegs = 168, kRegsIo = 72, kRegsSoftmax = 216;
 static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsIo <= kThreads * kLaunchRegs, "register split");
 constexpr float kLog2e = 1.4426950408889634f;
 
