@@ -568,7 +568,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
 #pragma unroll
                     for (int e = 0; e < 32; ++e) x[32 * c + e] = __uint_as_float(v[c][e]);
             };
-            load_s();
             const bool persistent = k < n_pt;
             const int lj = persistent ? 0 : k - n_pt;
             // valid-column masks of the tile (64 bits per half); recomputed where they are
@@ -603,19 +602,23 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                     if (!((mk1 >> c) & 1ull)) x[64 + c] = -CUDART_INF_F;
                 }
             };
-            if (masked) apply_mask();
             // Optimistic pass: the first half's exponentials against the running reference m
             // (what the lazy rescale uses whenever no row's maximum grew by more than 2^8),
             // with the tile's row maximum taken in the same pass.  Only when some row of the
             // warp needs a new reference (and always on the first tile) does the warp rescale
-            // O and l, reload S from TMEM (still intact: nothing is stored yet) and redo the
-            // first half.
+            // O and l and run the pass once more from S (still intact in TMEM: nothing is
+            // stored yet); the second pass never needs a new reference, and the loop keeps one
+            // copy of the pass in the code.
             float gs[16];
-            const float mu0 = (m == -CUDART_INF_F) ? 0.f : m;
-            const float mt = exp_half0_max(x, sl2, mu0, gs);
-            const float m_new = fmaxf(m, mt * sl2);
-            const bool need = m_new > m + 8.0f;
-            if (__any_sync(0xffffffffu, need)) {
+#pragma unroll 1
+            for (int pass = 0; pass < 2; ++pass) {
+                load_s();
+                if (masked) apply_mask();
+                const float mu0 = (m == -CUDART_INF_F) ? 0.f : m;
+                const float mt = exp_half0_max(x, sl2, mu0, gs);
+                const float m_new = fmaxf(m, mt * sl2);
+                const bool need = m_new > m + 8.0f;
+                if (!__any_sync(0xffffffffu, need)) break;
                 const float alpha = need ? fast_exp2(m - m_new) : 1.0f;
                 if (k > 0) {
                     if (!wwait(&bars[B_PV + X], (k - 1) & 1)) { ok = false; break; }
@@ -637,10 +640,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                     carry *= alpha;
                     m = m_new;
                 }
-                load_s();
-                if (masked) apply_mask();
-                exp_half<0>(x, sl2, (m == -CUDART_INF_F) ? 0.f : m, gs);
             }
+            if (!ok) break;
             const float mu = (m == -CUDART_INF_F) ? 0.f : m;
             // each half's P (bf16) goes over the first 64 columns of S as soon as it is done, so
             // the first store overlaps the second half's exponentials
